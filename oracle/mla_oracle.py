@@ -1,0 +1,235 @@
+"""CPU oracle for absorbed-MLA decode: plain, slow, fp64.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+CPU-baseline / reference arm may import this module; the library never does,
+and it shares no code with the CUDA path (the only common input is the seeded
+generator, which holds none of this arithmetic).
+
+What it computes, and where each step is defined:
+
+* Latent projection  c_t = W^DKV h_t                      -- "MLA deep compression"
+  (operatorworld.com), section on the low-rank projection (first equation).
+* Per-head up-projection  k^C_{t,i} = W^UK_i c_t,  v_{t,i} = W^UV_i c_t
+  -- same page and section, second equation.  The page prints the key matrix
+  as W^KR_i there; this oracle reads it as W^UK_i (the content-key
+  up-projection), because the same page later reserves W^KR for the RoPE key
+  projection from h, and "Attention-head anatomy" §5 names W^UK as the matrix
+  folded into the query path.
+* Decoupled RoPE  k^R_t = RoPE(W^KR h_t) shared by all heads,
+  q^R_i = RoPE(W^QR_i h), score = content dot product + RoPE dot product
+  -- "MLA deep compression", section on decoupled RoPE; "Attention-head
+  anatomy" §5 ("add the two dot products").  The pages give no RoPE
+  convention; this oracle uses rotations of consecutive pairs (2k, 2k+1) by
+  angle pos * base^(-2k/d_R).
+* Softmax over cached positions, o_i = sum_j a_ij v_{j,i}  -- "MLA deep
+  compression", section on absorption, output-side equation.
+* Absorption (for the separate absorbed helper and for checking the GPU's
+  intermediate u): W^QK_i = (W^UK_i)^T W^Q_i, score = (W^QK_i h)^T c,
+  u_i = sum_j a_ij c_j, o_i = W^UV_i u_i -- same section, both equations.
+* Cache width d_c + d_R and the KV-bytes formula 2*layers*kv_heads*head_dim*
+  bytes -- "MLA deep compression", decoupled-RoPE section; "Attention-head
+  anatomy" §2 and §4.
+
+Readings where the pages are silent: the softmax scale is a parameter; the
+s_q query rows of a sequence of length L sit at positions L - s_q + r and row
+r sees cached positions j <= L - s_q + r; lse is the natural log of
+sum_j exp(scale * s_j).
+
+Every function here is pinned by tests/test_oracle.py against brute force,
+closed forms and the figures the pages print.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+f64 = np.float64
+
+
+# ----------------------------------------------------------------------------
+# closed-form cache arithmetic
+# ----------------------------------------------------------------------------
+def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, bytes_per_elem: int) -> int:
+    """Per-token K/V cache bytes: 2 * layers * kv_heads * head_dim * bytes
+    ("Attention-head anatomy" §2, the one formula)."""
+    return 2 * layers * kv_heads * head_dim * bytes_per_elem
+
+
+def mla_cache_elems(d_c: int, d_R: int) -> int:
+    """Cached values per token per layer under MLA: the latent plus the shared
+    RoPE key ("MLA deep compression", decoupled-RoPE section)."""
+    return d_c + d_R
+
+
+def mha_kv_elems(n_h: int, d_h: int) -> int:
+    """K and V values per token per layer when every head caches its own pair
+    ("MLA deep compression", opening paragraph)."""
+    return 2 * n_h * d_h
+
+
+# ----------------------------------------------------------------------------
+# projections
+# ----------------------------------------------------------------------------
+def rope(x: np.ndarray, pos, base: float) -> np.ndarray:
+    """Rotate consecutive pairs (2k, 2k+1) of the last axis of x by angle
+    pos * base^(-2k/d).  ``pos`` broadcasts against x[..., 0]."""
+    x = np.asarray(x, dtype=f64)
+    d = x.shape[-1]
+    assert d % 2 == 0
+    k = np.arange(d // 2, dtype=f64)
+    theta = np.power(f64(base), -2.0 * k / d)                    # [d/2]
+    ang = np.asarray(pos, dtype=f64)[..., None] * theta           # [..., d/2]
+    cos, sin = np.cos(ang), np.sin(ang)
+    even, odd = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = even * cos - odd * sin
+    out[..., 1::2] = even * sin + odd * cos
+    return out
+
+
+def latent(W_DKV: np.ndarray, h: np.ndarray) -> np.ndarray:
+    """c = W^DKV h for every row of h: [..., d_model] -> [..., d_c]."""
+    return np.asarray(h, f64) @ np.asarray(W_DKV, f64).T
+
+
+def rope_key(W_KR: np.ndarray, h: np.ndarray, pos, base: float) -> np.ndarray:
+    """k^R = RoPE(W^KR h, pos): [..., d_model] -> [..., d_R]."""
+    return rope(np.asarray(h, f64) @ np.asarray(W_KR, f64).T, pos, base)
+
+
+def query_head(W_Q_i, W_QR_i, h, pos, base):
+    """Non-absorbed query of head i: [W^Q_i h || RoPE(W^QR_i h, pos)]."""
+    h = np.asarray(h, f64)
+    return np.concatenate([np.asarray(W_Q_i, f64) @ h,
+                           rope(np.asarray(W_QR_i, f64) @ h, pos, base)])
+
+
+def expanded_kv(C: np.ndarray, KR: np.ndarray, W_UK_i: np.ndarray, W_UV_i: np.ndarray):
+    """Per-head keys K_i = [W^UK_i c_j || k^R_j] and values V_i = W^UV_i c_j for
+    every cached row j: C [L, d_c], KR [L, d_R] -> K [L, d_h + d_R], V [L, d_v]."""
+    C = np.asarray(C, f64)
+    K = np.concatenate([C @ np.asarray(W_UK_i, f64).T, np.asarray(KR, f64)], axis=1)
+    V = C @ np.asarray(W_UV_i, f64).T
+    return K, V
+
+
+def softmax_attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float, n_valid: int):
+    """a = softmax(scale * K q) over rows j < n_valid; returns (a V, lse, a)."""
+    s = scale * (np.asarray(K[:n_valid], f64) @ np.asarray(q, f64))
+    m = s.max()
+    e = np.exp(s - m)
+    z = e.sum()
+    a = e / z
+    return a @ np.asarray(V[:n_valid], f64), m + math.log(z), a
+
+
+# ----------------------------------------------------------------------------
+# cache access
+# ----------------------------------------------------------------------------
+def gather_rows(cache, block_table, page_size: int, b: int, L: int):
+    """Logical rows 0..L-1 of sequence b through its block table."""
+    j = np.arange(L)
+    rows = np.asarray(block_table)[b, j // page_size].astype(np.int64) * page_size + j % page_size
+    return np.asarray(cache, f64)[rows]
+
+
+def pipeline_cache(inp: dict, w) -> np.ndarray:
+    """The cache a full-pipeline workload holds: row of position t of sequence
+    b is [W^DKV h_t || RoPE(W^KR h_t, t)], stored through the block table."""
+    rows = inp["num_pages"] * w.page_size
+    cache = np.zeros((rows, w.d_c + w.d_R), dtype=f64)
+    for b in range(w.B):
+        L = int(inp["seqlens"][b])
+        h = np.asarray(inp["h_ctx"][b, :L], f64)
+        t = np.arange(L)
+        rid = np.asarray(inp["block_table"])[b, t // w.page_size].astype(np.int64) * w.page_size + t % w.page_size
+        cache[rid, :w.d_c] = latent(inp["W_DKV"], h)
+        cache[rid, w.d_c:] = rope_key(inp["W_KR"], h, t, w.rope_base)
+    return cache
+
+
+def _cache_of(inp, w):
+    return inp["cache"] if "cache" in inp else pipeline_cache(inp, w)
+
+
+# ----------------------------------------------------------------------------
+# decode, expanded (the definition)
+# ----------------------------------------------------------------------------
+def decode_expanded(inp: dict, w, picks=None, cache=None):
+    """Non-absorbed decode.
+
+    For every picked (b, r, i): materialise K_i and V_i for the cached rows of
+    sequence b, form q_i from h, mask positions j > L_b - s_q + r, softmax,
+    and take o = sum_j a_j v_j.  Returns dict (b, r, i) -> (o [d_v], lse).
+    ``picks`` None means every (b, r, i).
+    """
+    cache = _cache_of(inp, w) if cache is None else cache
+    if picks is None:
+        picks = [(b, r, i) for b in range(w.B) for r in range(w.s_q) for i in range(w.n_h)]
+    by_seq = {}
+    for (b, r, i) in picks:
+        by_seq.setdefault(b, []).append((r, i))
+    out = {}
+    for b, items in by_seq.items():
+        L = int(inp["seqlens"][b])
+        rows = gather_rows(cache, inp["block_table"], w.page_size, b, L)
+        C, KR = rows[:, :w.d_c], rows[:, w.d_c:]
+        heads = sorted({i for _, i in items})
+        kv = {i: expanded_kv(C, KR, inp["W_UK"][i], inp["W_UV"][i]) for i in heads}
+        for (r, i) in items:
+            pos = int(inp["qpos"][b, r])
+            q = query_head(inp["W_Q"][i], inp["W_QR"][i], inp["h_q"][b, r], pos, w.rope_base)
+            K, V = kv[i]
+            o, lse, _ = softmax_attend(q, K, V, w.softmax_scale, n_valid=pos + 1)
+            out[(b, r, i)] = (o, lse)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# absorbed helper (separate code path, used to check the GPU's u)
+# ----------------------------------------------------------------------------
+def absorb_weights(W_UK: np.ndarray, W_Q: np.ndarray) -> np.ndarray:
+    """W^QK_i = (W^UK_i)^T W^Q_i: [n_h, d_h, d_c] x [n_h, d_h, d_model] -> [n_h, d_c, d_model]."""
+    return np.einsum("hkc,hkd->hcd", np.asarray(W_UK, f64), np.asarray(W_Q, f64))
+
+
+def absorbed_query(inp: dict, w, b: int, r: int, i: int, W_QK_i=None) -> np.ndarray:
+    """q^lat_i = W^QK_i h (or W^UK_i^T (W^Q_i h) when W^QK_i is not given),
+    concatenated with q^R_i = RoPE(W^QR_i h, pos): [d_c + d_R]."""
+    h = np.asarray(inp["h_q"][b, r], f64)
+    if W_QK_i is None:
+        qlat = np.asarray(inp["W_UK"][i], f64).T @ (np.asarray(inp["W_Q"][i], f64) @ h)
+    else:
+        qlat = np.asarray(W_QK_i, f64) @ h
+    qr = rope(np.asarray(inp["W_QR"][i], f64) @ h, int(inp["qpos"][b, r]), w.rope_base)
+    return np.concatenate([qlat, qr])
+
+
+def decode_absorbed(q: np.ndarray, cache, block_table, seqlens, w, picks=None):
+    """Absorbed decode from an explicit query tensor q [B, s_q, n_h, d_c + d_R]:
+    s_j = q^lat.c_j + q^R.k^R_j, a = softmax(scale s) over j <= L - s_q + r,
+    u = sum_j a_j c_j.  Returns dict (b, r, i) -> (u [d_c], lse)."""
+    if picks is None:
+        picks = [(b, r, i) for b in range(w.B) for r in range(w.s_q) for i in range(w.n_h)]
+    by_seq = {}
+    for (b, r, i) in picks:
+        by_seq.setdefault(b, []).append((r, i))
+    out = {}
+    for b, items in by_seq.items():
+        L = int(seqlens[b])
+        rows = gather_rows(cache, block_table, w.page_size, b, L)
+        for (r, i) in items:
+            n_valid = L - w.s_q + r + 1
+            qv = np.asarray(q[b, r, i], f64)
+            s = w.softmax_scale * (rows[:n_valid] @ qv)
+            m = s.max()
+            e = np.exp(s - m)
+            z = e.sum()
+            out[(b, r, i)] = ((e / z) @ rows[:n_valid, :w.d_c], m + math.log(z))
+    return out
+
+
+def up_project(u: np.ndarray, W_UV: np.ndarray) -> np.ndarray:
+    """o_i = W^UV_i u_i: u [..., n_h, d_c], W^UV [n_h, d_v, d_c] -> [..., n_h, d_v]."""
+    return np.einsum("...hc,hvc->...hv", np.asarray(u, f64), np.asarray(W_UV, f64))
