@@ -1,0 +1,194 @@
+/*
+ * libmla -- absorbed Multi-head Latent Attention (MLA) decode for B200 (sm_100a).
+ *
+ * The math (sources named by page title and section):
+ *   - "MLA deep compression" (operatorworld.com), absorption section, score
+ *     equation: head i scores the cached latent c directly with the absorbed
+ *     query q^lat_i = W^QK_i h, where W^QK_i = (W^UK_i)^T W^Q_i is formed
+ *     offline once per model.
+ *   - same page, absorption section, output equation: o_i = W^UV_i u_i with
+ *     u_i = sum_j a_ij c_j, the softmax-weighted sum of cached latents.
+ *   - same page, decoupled-RoPE section: each cached row also holds a 64-wide
+ *     RoPE key k^R shared by all heads; the score adds q^R_i . k^R_j to the
+ *     latent dot product, so a cached row is [c (d_c) || k^R (d_R)], 576
+ *     values at the DeepSeek-V3 shape.
+ *   - "Attention-head anatomy" (romaanj.github.io) section 5: the same fold
+ *     of W^UK into the query path and the sum of the two dot products.
+ *
+ * Conventions for every call:
+ *   - Pointers named as device buffers are device pointers the caller owns;
+ *     the library allocates nothing and frees nothing.  Scratch space for
+ *     mla_decode is passed in as `workspace`.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream; arguments are
+ *     validated on the host first and a non-OK status means nothing was
+ *     enqueued.  A launch failure reported by the CUDA runtime returns
+ *     MLA_ERR_CUDA.
+ *   - Element type is chosen by `dtype`: MLA_DTYPE_BF16 tensors hold bf16,
+ *     MLA_DTYPE_FP32 tensors hold fp32.  Index tensors are int32.  Softmax
+ *     statistics (lse) are always fp32.  Accumulation is always fp32.
+ *   - All tensors are dense row-major with the shapes given; every device
+ *     pointer must be 16-byte aligned.
+ *   - Problems the host cannot see (a sequence length or page id out of
+ *     range in device memory, a device-side wait that ran out of time) set a
+ *     sticky device flag instead of faulting; mla_check_device_errors reads
+ *     and clears it.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,          /* null/unaligned pointer, bad size, bad dtype */
+  MLA_ERR_UNSUPPORTED = 2,          /* valid but not implemented (e.g. n_h > 128) */
+  MLA_ERR_CUDA = 3,                 /* CUDA runtime/driver error */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < mla_decode_workspace_size */
+  MLA_ERR_DEVICE_CHECK = 5          /* device flag raised (see mla_check_device_errors) */
+} mla_status;
+
+typedef enum { MLA_DTYPE_BF16 = 0, MLA_DTYPE_FP32 = 1 } mla_dtype;
+
+/* Device flag bits reported by mla_check_device_errors (OR-ed together). */
+#define MLA_DEVFLAG_BAD_SEQLEN 0x1  /* seqlens[b] < s_q or > max_pages_per_seq*page_size */
+#define MLA_DEVFLAG_BAD_PAGE 0x2    /* block_table entry outside [0, num_pages) */
+#define MLA_DEVFLAG_TIMEOUT 0x4     /* a device-side wait gave up (kernel returned early) */
+
+const char* mla_status_string(mla_status s);
+
+/*
+ * Offline weight absorption, score side ("MLA deep compression", absorption
+ * section, score equation):  W_QK[i] = W_UK[i]^T . W_Q[i]  for every head i.
+ *   W_UK  [n_h, d_h, d_c]      device, read
+ *   W_Q   [n_h, d_h, d_model]  device, read
+ *   W_QK  [n_h, d_c, d_model]  device, written
+ * Run once per model; not on the per-token path.
+ */
+mla_status mla_absorb_weights(const void* W_UK, const void* W_Q, void* W_QK, int n_h, int d_h,
+                              int d_c, int d_model, mla_dtype dtype, void* stream);
+
+/*
+ * Absorbed query formation ("MLA deep compression", absorption section score
+ * equation and decoupled-RoPE section):
+ *   q[t, i, 0:d_c]       = W_QK[i] . h[t]
+ *   q[t, i, d_c:d_c+d_R] = RoPE(W_QR[i] . h[t], pos[t])
+ * RoPE rotates consecutive pairs (2k, 2k+1) by angle pos * rope_base^(-2k/d_R)
+ * (the pages give no convention; this is the plain rotary one).
+ *   h     [T, d_model]             device, read
+ *   W_QK  [n_h, d_c, d_model]      device, read (from mla_absorb_weights)
+ *   W_QR  [n_h, d_R, d_model]      device, read
+ *   pos   [T] int32                device, read (query positions)
+ *   q     [T, n_h, d_c + d_R]      device, written (T = B * s_q rows)
+ */
+mla_status mla_form_query(const void* h, const void* W_QK, const void* W_QR, const int* pos,
+                          void* q, int T, int n_h, int d_model, int d_c, int d_R, float rope_base,
+                          mla_dtype dtype, void* stream);
+
+/*
+ * Latent append ("MLA deep compression", low-rank projection section and
+ * decoupled-RoPE section): for each new token t of sequence seq_ids[t] at
+ * position pos[t], writes the cache row
+ *   kv_cache[row] = [ W_DKV . h[t]  ||  RoPE(W_KR . h[t], pos[t]) ]
+ * where row = block_table[seq_ids[t]][pos[t] / page_size] * page_size + pos[t] % page_size.
+ *   h           [T, d_model]                      device, read
+ *   W_DKV       [d_c, d_model]                    device, read
+ *   W_KR        [d_R, d_model]                    device, read
+ *   seq_ids,pos [T] int32                         device, read
+ *   block_table [*, max_pages_per_seq] int32      device, read
+ *   kv_cache    [num_pages*page_size, d_c + d_R]  device, written (only the T rows)
+ * Out-of-range page ids raise MLA_DEVFLAG_BAD_PAGE and the row is skipped.
+ */
+mla_status mla_append_latent(const void* h, const void* W_DKV, const void* W_KR,
+                             const int* seq_ids, const int* pos, const int* block_table,
+                             int max_pages_per_seq, int page_size, int num_pages, void* kv_cache,
+                             int T, int d_model, int d_c, int d_R, float rope_base,
+                             mla_dtype dtype, void* stream);
+
+/*
+ * Absorbed decode over a paged latent cache ("MLA deep compression",
+ * absorption section, both equations; decoupled-RoPE section):
+ *   for every sequence b, query row r < s_q, head i:
+ *     s_j  = q[b,r,i,:d_c] . c_j + q[b,r,i,d_c:] . kR_j     for j <= seqlens[b] - s_q + r
+ *     a    = softmax(softmax_scale * s)
+ *     u[b,r,i,:]  = sum_j a_j c_j
+ *     lse[b,r,i]  = log(sum_j exp(softmax_scale * s_j))      (natural log)
+ * The s_q query rows are the last s_q positions of the sequence (already in
+ * the cache); row r sees every cached position up to and including its own.
+ * Long or ragged contexts are cut into KV chunks that run in parallel and are
+ * merged by a combine step (log-sum-exp weighting).
+ */
+typedef struct {
+  const void* q;            /* [B, s_q, n_h, d_c + d_R] device; latent part first, then RoPE   */
+  const void* kv_cache;     /* [num_pages * page_size, d_c + d_R] device; row = c || k^R        */
+  const int* block_table;   /* [B, max_pages_per_seq] int32 device; physical page ids          */
+  const int* seqlens;       /* [B] int32 device; cached tokens incl. the s_q query tokens        */
+  void* u;                  /* [B, s_q, n_h, d_c] device, written                                */
+  float* lse;               /* [B, s_q, n_h] fp32 device, written; may be NULL                   */
+  int B;                    /* sequences; 0 is a no-op                                           */
+  int s_q;                  /* query rows per sequence: 1 or 2                                   */
+  int n_h;                  /* heads, 1..128                                                     */
+  int d_c;                  /* latent width (512 at the DeepSeek-V3 shape), multiple of 8, <=512 */
+  int d_R;                  /* RoPE key width (64), even, multiple of 8 with d_c, <= 64          */
+  int page_size;            /* tokens per page, a positive multiple of 64                         */
+  int max_pages_per_seq;    /* columns of block_table                                            */
+  int num_pages;            /* pages in kv_cache                                                 */
+  float softmax_scale;      /* multiplies the scores before softmax, finite                       */
+  mla_dtype dtype;          /* of q, kv_cache and u                                              */
+  int num_splits;           /* KV chunks the whole batch is cut into; 0 = one per SM pair        */
+} mla_decode_params;
+
+/* Bytes of device scratch mla_decode needs for these parameters (depends on
+ * B, s_q, n_h, d_c, num_splits and the current device's SM count). */
+mla_status mla_decode_workspace_size(const mla_decode_params* p, size_t* bytes);
+
+/* Runs plan + attend + combine.  `workspace` must be 256-byte aligned device
+ * memory of at least mla_decode_workspace_size bytes; it is scratch (no
+ * state is kept between calls).  Rows of a page past seqlens[b] may hold
+ * any bit pattern (they are never used).  Calls that share a workspace must
+ * be ordered on the GPU. */
+mla_status mla_decode(const mla_decode_params* p, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* The three stages of mla_decode, for callers that time or schedule them
+ * separately; calling them in this order is exactly mla_decode.
+ *   plan:    per-sequence tile counts and KV-chunk boundaries into the workspace
+ *   attend:  the chunked attention (writes u/lse directly for unsplit rows,
+ *            fp32 partials into the workspace otherwise)
+ *   combine: merges the partials of split rows into u/lse */
+mla_status mla_decode_plan(const mla_decode_params* p, void* workspace, size_t workspace_bytes,
+                           void* stream);
+mla_status mla_decode_attend(const mla_decode_params* p, void* workspace, size_t workspace_bytes,
+                             void* stream);
+mla_status mla_decode_combine(const mla_decode_params* p, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Which attend kernel these parameters select: 1 = tensor-core (tcgen05)
+ * kernel, 0 = CUDA-core kernel; and the number of KV chunks it will use. */
+mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_cores,
+                                  int* num_chunks);
+
+/*
+ * Per-head up-projection ("MLA deep compression", absorption section, output
+ * equation):  o[t, i, :] = W_UV[i] . u[t, i, :]
+ *   u     [T, n_h, d_c]   device, read   (T = B * s_q)
+ *   W_UV  [n_h, d_v, d_c] device, read
+ *   o     [T, n_h, d_v]   device, written
+ */
+mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c,
+                       int d_v, mla_dtype dtype, void* stream);
+
+/* Synchronizes `stream`, then reads and clears the device flag of the
+ * current device.  Returns MLA_OK if no flag was raised, otherwise
+ * MLA_ERR_DEVICE_CHECK and the MLA_DEVFLAG_* bits in *flags (may be NULL). */
+mla_status mla_check_device_errors(void* stream, int* flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

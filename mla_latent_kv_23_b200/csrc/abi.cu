@@ -1,0 +1,474 @@
+// C ABI of libmla: argument validation, workspace sizing, TMA descriptor
+// encoding and kernel selection.  No allocation happens here: every device
+// buffer, the workspace included, belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "mla.h"
+
+namespace mla {
+
+// Sticky device-side flags (MLA_DEVFLAG_*), one word per device.
+__device__ int g_device_flags;
+
+int decode_sm100_prepare();
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  int max_clusters = 0;  // co-resident 2-CTA clusters of the tensor-core kernel
+  int* flags = nullptr;  // device address of g_device_flags
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+mla_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MLA_OK;
+  cudaGetLastError();
+  return MLA_ERR_CUDA;
+}
+
+mla_status device_info(const DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready) {
+    cudaError_t e;
+    if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_status(e);
+    if ((e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_status(e);
+    if ((e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_status(e);
+    if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.flags), g_device_flags)) != cudaSuccess)
+      return cuda_status(e);
+    d.max_clusters = (d.cc_major == 10) ? decode_sm100_prepare() : 0;
+    if (g_encode == nullptr) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+              cudaSuccess &&
+          q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      cudaGetLastError();
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return MLA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(mla_dtype d) { return d == MLA_DTYPE_BF16 || d == MLA_DTYPE_FP32; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+mla_status validate_decode(const mla_decode_params* p) {
+  if (p == nullptr) return MLA_ERR_INVALID_ARG;
+  if (p->B < 0) return MLA_ERR_INVALID_ARG;
+  if (p->s_q < 1) return MLA_ERR_INVALID_ARG;
+  if (p->s_q > 2) return MLA_ERR_UNSUPPORTED;
+  if (p->n_h < 1) return MLA_ERR_INVALID_ARG;
+  if (p->n_h > kMaxHeads) return MLA_ERR_UNSUPPORTED;
+  if (p->d_c < 8 || p->d_c % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (p->d_c > 512) return MLA_ERR_UNSUPPORTED;
+  if (p->d_R < 0 || p->d_R % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (p->d_R > 64) return MLA_ERR_UNSUPPORTED;
+  if (p->page_size <= 0 || p->page_size % kTileTokens != 0) return MLA_ERR_INVALID_ARG;
+  if (p->max_pages_per_seq < 1 || p->num_pages < 1) return MLA_ERR_INVALID_ARG;
+  if ((long long)p->num_pages * p->page_size > INT_MAX) return MLA_ERR_UNSUPPORTED;
+  if ((long long)p->max_pages_per_seq * p->page_size > INT_MAX) return MLA_ERR_UNSUPPORTED;
+  if (!std::isfinite(p->softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!valid_dtype(p->dtype)) return MLA_ERR_INVALID_ARG;
+  if (p->num_splits < 0) return MLA_ERR_INVALID_ARG;
+  if (p->B == 0) return MLA_OK;
+  if ((long long)p->B * p->s_q * p->n_h > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  if (!p->q || !p->kv_cache || !p->block_table || !p->seqlens || !p->u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(p->q) || !aligned16(p->kv_cache) || !aligned16(p->u) ||
+      !aligned16(p->block_table) || !aligned16(p->seqlens) || (p->lse && !aligned16(p->lse)))
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+bool use_tensor_cores(const mla_decode_params* p, const DeviceInfo* d) {
+  return d->cc_major == 10 && d->max_clusters > 0 && p->dtype == MLA_DTYPE_BF16 && p->d_c == 512 &&
+         p->d_R == 64 && g_encode != nullptr;
+}
+
+int choose_chunks(const mla_decode_params* p, const DeviceInfo* d) {
+  if (p->num_splits > 0) return p->num_splits;
+  if (use_tensor_cores(p, d)) return std::max(1, d->max_clusters / p->s_q);
+  return std::max(1, (2 * d->sm_count) / (p->s_q * p->n_h));
+}
+
+struct Resolved {
+  DecodeArgs a;
+  bool tc = false;
+  const DeviceInfo* dev = nullptr;
+};
+
+mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolved* r) {
+  mla_status st = validate_decode(p);
+  if (st != MLA_OK) return st;
+  if ((st = device_info(&r->dev)) != MLA_OK) return st;
+  const int G = choose_chunks(p, r->dev);
+  if ((long long)G * p->s_q * 2 > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  const WsLayout L = ws_layout(p->B, p->s_q, p->n_h, p->d_c, G);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MLA_ERR_INVALID_ARG;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  DecodeArgs& a = r->a;
+  a.q = p->q;
+  a.kv = p->kv_cache;
+  a.block_table = p->block_table;
+  a.seqlens = p->seqlens;
+  a.u = p->u;
+  a.lse = p->lse;
+  a.header = reinterpret_cast<int*>(w + L.header);
+  a.tile_prefix = reinterpret_cast<int*>(w + L.tile_prefix);
+  a.split_base = reinterpret_cast<int*>(w + L.split_base);
+  a.part_lse = reinterpret_cast<float*>(w + L.part_lse);
+  a.part_u = reinterpret_cast<float*>(w + L.part_u);
+  a.err = r->dev->flags;
+  a.B = p->B;
+  a.s_q = p->s_q;
+  a.n_h = p->n_h;
+  a.d_c = p->d_c;
+  a.d_R = p->d_R;
+  a.page_size = p->page_size;
+  a.max_pages = p->max_pages_per_seq;
+  a.num_pages = p->num_pages;
+  a.num_chunks = G;
+  a.scale = p->softmax_scale;
+  a.bf16 = p->dtype == MLA_DTYPE_BF16;
+  r->tc = use_tensor_cores(p, r->dev);
+  return MLA_OK;
+}
+
+mla_status encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_x,
+                     uint32_t box_y, CUtensorMapSwizzle sw) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_x, box_y};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s) {
+  if (!r.tc) return cuda_status(launch_decode_simt(r.a, s));
+  Sm100Maps maps;
+  const uint64_t qrows = (uint64_t)p->B * p->s_q * p->n_h;
+  const uint64_t kvrows = (uint64_t)p->num_pages * p->page_size;
+  mla_status st;
+  if ((st = encode_2d(&maps.q_lat, p->q, 576, qrows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+      (st = encode_2d(&maps.q_rope, p->q, 576, qrows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK ||
+      (st = encode_2d(&maps.kv_lat, p->kv_cache, 576, kvrows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+      (st = encode_2d(&maps.kv_rope, p->kv_cache, 576, kvrows, 32, 64, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+    return st;
+  return cuda_status(launch_decode_sm100(r.a, maps, s));
+}
+
+}  // namespace
+
+WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks) {
+  WsLayout L;
+  L.slots = (long long)(B + num_chunks) * s_q;
+  size_t off = 0;
+  L.header = off;
+  off += 256;
+  L.tile_prefix = off;
+  off = align_up(off + sizeof(int) * (B + 1), 256);
+  L.split_base = off;
+  off = align_up(off + sizeof(int) * (B + 1), 256);
+  L.part_lse = off;
+  off = align_up(off + sizeof(float) * (size_t)L.slots * n_h, 256);
+  L.part_u = off;
+  off = align_up(off + sizeof(float) * (size_t)L.slots * n_h * d_c, 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MLA_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+mla_status mla_decode_workspace_size(const mla_decode_params* p, size_t* bytes) {
+  if (bytes == nullptr) return MLA_ERR_INVALID_ARG;
+  mla_status st = validate_decode(p);
+  if (st != MLA_OK) return st;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  *bytes = ws_layout(p->B, p->s_q, p->n_h, p->d_c, choose_chunks(p, d)).total;
+  return MLA_OK;
+}
+
+mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_cores,
+                                  int* num_chunks) {
+  mla_status st = validate_decode(p);
+  if (st != MLA_OK) return st;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  if (uses_tensor_cores) *uses_tensor_cores = use_tensor_cores(p, d) ? 1 : 0;
+  if (num_chunks) *num_chunks = choose_chunks(p, d);
+  return MLA_OK;
+}
+
+mla_status mla_decode_plan(const mla_decode_params* p, void* ws, size_t ws_bytes, void* stream) {
+  if (p != nullptr && p->B == 0) return validate_decode(p);
+  Resolved r;
+  mla_status st = resolve(p, ws, ws_bytes, &r);
+  if (st != MLA_OK) return st;
+  return cuda_status(launch_plan(r.a, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_decode_attend(const mla_decode_params* p, void* ws, size_t ws_bytes, void* stream) {
+  if (p != nullptr && p->B == 0) return validate_decode(p);
+  Resolved r;
+  mla_status st = resolve(p, ws, ws_bytes, &r);
+  if (st != MLA_OK) return st;
+  return attend(r, p, static_cast<cudaStream_t>(stream));
+}
+
+mla_status mla_decode_combine(const mla_decode_params* p, void* ws, size_t ws_bytes, void* stream) {
+  if (p != nullptr && p->B == 0) return validate_decode(p);
+  Resolved r;
+  mla_status st = resolve(p, ws, ws_bytes, &r);
+  if (st != MLA_OK) return st;
+  return cuda_status(launch_combine(r.a, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_decode(const mla_decode_params* p, void* ws, size_t ws_bytes, void* stream) {
+  if (p != nullptr && p->B == 0) return validate_decode(p);
+  Resolved r;
+  mla_status st = resolve(p, ws, ws_bytes, &r);
+  if (st != MLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
+  if ((st = attend(r, p, s)) != MLA_OK) return st;
+  return cuda_status(launch_combine(r.a, s));
+}
+
+mla_status mla_absorb_weights(const void* W_UK, const void* W_Q, void* W_QK, int n_h, int d_h,
+                              int d_c, int d_model, mla_dtype dtype, void* stream) {
+  if (!W_UK || !W_Q || !W_QK || !valid_dtype(dtype)) return MLA_ERR_INVALID_ARG;
+  if (n_h < 1 || d_h < 1 || d_c < 1 || d_model < 1) return MLA_ERR_INVALID_ARG;
+  if (n_h > 65535) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(W_UK) || !aligned16(W_Q) || !aligned16(W_QK)) return MLA_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  GemmArgs g = {};
+  g.A = W_UK;  // A(z, m = c, k) = W_UK[z][k][c]
+  g.Bm = W_Q;  // B(z, n = d, k) = W_Q[z][k][d]
+  g.C = W_QK;
+  g.M = d_c;
+  g.N = d_model;
+  g.K = d_h;
+  g.Z = n_h;
+  g.sAz = (long long)d_h * d_c;
+  g.sAm = 1;
+  g.sAk = d_c;
+  g.sBz = (long long)d_h * d_model;
+  g.sBn = 1;
+  g.sBk = d_model;
+  g.sCz = (long long)d_c * d_model;
+  g.sCm = d_model;
+  g.seg = INT_MAX;
+  g.err = d->flags;
+  g.bf16 = dtype == MLA_DTYPE_BF16;
+  return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_form_query(const void* h, const void* W_QK, const void* W_QR, const int* pos,
+                          void* q, int T, int n_h, int d_model, int d_c, int d_R, float rope_base,
+                          mla_dtype dtype, void* stream) {
+  if (!valid_dtype(dtype) || T < 0 || n_h < 1 || d_model < 1 || d_c < 1 || d_R < 0 || d_R % 2)
+    return MLA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !W_QK || !q || (d_R > 0 && (!W_QR || !pos))) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(W_QK) || !aligned16(q) || (W_QR && !aligned16(W_QR)))
+    return MLA_ERR_INVALID_ARG;
+  if (T > 65535 * 64) return MLA_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int W = d_c + d_R;
+  GemmArgs g = {};
+  g.A = h;
+  g.M = T;
+  g.K = d_model;
+  g.Z = 1;
+  g.sAm = d_model;
+  g.sAk = 1;
+  g.sBk = 1;
+  g.sBn = d_model;
+  g.sCm = (long long)n_h * W;
+  g.err = d->flags;
+  g.bf16 = dtype == MLA_DTYPE_BF16;
+  // latent part: n = i * d_c + c
+  g.Bm = W_QK;
+  g.C = q;
+  g.N = n_h * d_c;
+  g.seg = d_c;
+  g.seg_stride = W;
+  g.col_off = 0;
+  if ((st = cuda_status(launch_gemm(g, s))) != MLA_OK) return st;
+  if (d_R == 0) return MLA_OK;
+  // RoPE part: n = i * d_R + k, rotated by the query position
+  g.Bm = W_QR;
+  g.N = n_h * d_R;
+  g.seg = d_R;
+  g.seg_stride = W;
+  g.col_off = d_c;
+  g.pos = pos;
+  g.rope = 1;
+  g.rope_base = rope_base;
+  return cuda_status(launch_gemm(g, s));
+}
+
+mla_status mla_append_latent(const void* h, const void* W_DKV, const void* W_KR,
+                             const int* seq_ids, const int* pos, const int* block_table,
+                             int max_pages_per_seq, int page_size, int num_pages, void* kv_cache,
+                             int T, int d_model, int d_c, int d_R, float rope_base,
+                             mla_dtype dtype, void* stream) {
+  if (!valid_dtype(dtype) || T < 0 || d_model < 1 || d_c < 1 || d_R < 0 || d_R % 2 ||
+      page_size < 1 || max_pages_per_seq < 1 || num_pages < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !W_DKV || !seq_ids || !pos || !block_table || !kv_cache || (d_R > 0 && !W_KR))
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(kv_cache) || (W_KR && !aligned16(W_KR)))
+    return MLA_ERR_INVALID_ARG;
+  if (T > 65535 * 64) return MLA_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemmArgs g = {};
+  g.A = h;
+  g.C = kv_cache;
+  g.M = T;
+  g.K = d_model;
+  g.Z = 1;
+  g.sAm = d_model;
+  g.sAk = 1;
+  g.sBn = d_model;
+  g.sBk = 1;
+  g.sCm = d_c + d_R;
+  g.seg = INT_MAX;
+  g.pos = pos;
+  g.seq = seq_ids;
+  g.block_table = block_table;
+  g.max_pages = max_pages_per_seq;
+  g.page_size = page_size;
+  g.num_pages = num_pages;
+  g.err = d->flags;
+  g.bf16 = dtype == MLA_DTYPE_BF16;
+  g.Bm = W_DKV;
+  g.N = d_c;
+  g.col_off = 0;
+  if ((st = cuda_status(launch_gemm(g, s))) != MLA_OK) return st;
+  if (d_R == 0) return MLA_OK;
+  g.Bm = W_KR;
+  g.N = d_R;
+  g.col_off = d_c;
+  g.seg = d_R;
+  g.seg_stride = 0;
+  g.rope = 1;
+  g.rope_base = rope_base;
+  return cuda_status(launch_gemm(g, s));
+}
+
+mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c, int d_v,
+                       mla_dtype dtype, void* stream) {
+  if (!valid_dtype(dtype) || T < 0 || n_h < 1 || d_c < 1 || d_v < 1) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!u || !W_UV || !o) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(W_UV) || !aligned16(o)) return MLA_ERR_INVALID_ARG;
+  if (n_h > 65535 || T > 65535 * 64) return MLA_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  GemmArgs g = {};
+  g.A = u;     // A(z = head, m = t, k = c) = u[t][z][c]
+  g.Bm = W_UV; // B(z, n = v, k = c) = W_UV[z][v][c]
+  g.C = o;     // C(z, m = t, n = v) = o[t][z][v]
+  g.M = T;
+  g.N = d_v;
+  g.K = d_c;
+  g.Z = n_h;
+  g.sAz = d_c;
+  g.sAm = (long long)n_h * d_c;
+  g.sAk = 1;
+  g.sBz = (long long)d_v * d_c;
+  g.sBn = d_c;
+  g.sBk = 1;
+  g.sCz = d_v;
+  g.sCm = (long long)n_h * d_v;
+  g.seg = INT_MAX;
+  g.err = d->flags;
+  g.bf16 = dtype == MLA_DTYPE_BF16;
+  return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_check_device_errors(void* stream, int* flags) {
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  int v = 0;
+  if ((e = cudaMemcpy(&v, d->flags, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_status(e);
+  if (v != 0) {
+    const int zero = 0;
+    if ((e = cudaMemcpy(d->flags, &zero, sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
+      return cuda_status(e);
+  }
+  if (flags) *flags = v;
+  return v == 0 ? MLA_OK : MLA_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

@@ -1,0 +1,518 @@
+// Attend stage on the 5th-generation tensor cores (sm_100a), for n_h <= 128
+// heads, latent d_c = 512, RoPE key d_R = 64, bf16.
+//
+// Math ("MLA deep compression", absorption section, both equations, and its
+// decoupled-RoPE section): all heads of one query row share every cached row
+// [c || k^R], so the 128 heads are the M dimension of two dense contractions
+// per 64-token tile:
+//     S = Q . [C || K^R]^T      (M = 128, N = 64 tokens, K = 576)
+//     O = O * alpha + P . C     (M = 128, N = 512 latent, K = 64 tokens)
+// with an online softmax between them; u = O / l at the end.
+//
+// Layout.  O for 128 heads x 512 latent in fp32 fills all 512 TMEM columns,
+// which leaves no room for S.  So a cluster of two CTAs splits the columns:
+// CTA r owns latent columns [256r, 256r + 256) and RoPE columns
+// [32r, 32r + 32).  Each CTA loads only its own columns of every cache tile
+// (each byte is read from HBM once), computes a partial S over its 288
+// columns, and the two partial S tiles are exchanged through distributed
+// shared memory.  Both CTAs then hold the same S (fp32 addition commutes),
+// make bit-identical softmax decisions, and each accumulates its own half of
+// O = P . C (N = 256).  TMEM per CTA: O 256 columns + 2 S buffers of 64.
+//
+// One shared-memory tile serves both contractions: a TMA load with 128-byte
+// swizzle writes each 64-column block as 64 rows x 128 B, which is the
+// K-major operand layout of S = Q K^T and the MN-major operand layout of
+// O = P C at the same time.
+//
+// Warp roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and
+// zeroes cache rows past the end of a sequence), warp 2 = TMEM allocator,
+// warps 4-7 = softmax / correction / epilogue, one thread per head (TMEM lane).
+//
+// Work: the plan stage cuts the batch's tiles into equal chunks; cluster c
+// handles chunk c / s_q for query row c % s_q, walking its segments in order.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+#include "schedule.cuh"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace {
+using namespace ptx;
+
+constexpr int kThreads = 256;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpAlloc = 2, kWarpSoftmax0 = 4;
+constexpr int kStages = 2;
+constexpr int kDc = 512;
+constexpr int kLatPerCta = 256, kRopePerCta = 32;
+
+constexpr uint32_t kQBlk = 128 * 128;                    // Q: 128 rows x 64 cols bf16, SW128
+constexpr uint32_t kQRope = 128 * 64;                    // Q: 128 rows x 32 cols bf16, SW64
+constexpr uint32_t kQBytes = 4 * kQBlk + kQRope;         // 73728
+constexpr uint32_t kKvBlk = 64 * 128;                    // tile: 64 rows x 64 cols, SW128
+constexpr uint32_t kKvRope = 64 * 64;                    // tile: 64 rows x 32 cols, SW64
+constexpr uint32_t kStageBytes = 4 * kKvBlk + kKvRope;   // 36864
+constexpr uint32_t kPBytes = 128 * 128;                  // P: 128 rows x 64 tokens bf16, SW128
+constexpr uint32_t kXBytes = 128 * 256;                  // peer partial S: 128 x 64 fp32
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKv = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;
+constexpr uint32_t kOffX = kOffP + kPBytes;
+constexpr uint32_t kOffBar = kOffX + kXBytes;
+
+enum Bar {
+  KV_FULL = 0,
+  KV_EMPTY = KV_FULL + kStages,
+  S_FULL = KV_EMPTY + kStages,
+  S_EMPTY = S_FULL + 2,
+  P_FULL = S_EMPTY + 2,
+  PV_DONE,
+  X_FULL,
+  X_EMPTY,
+  Q_FULL,
+  Q_EMPTY,
+  MMA_FINAL,
+  BAR_COUNT
+};
+constexpr uint32_t kOffTmemSlot = kOffBar + BAR_COUNT * 8;
+constexpr uint32_t kSmemUsed = kOffTmemSlot + 16;
+constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 0;     // 256 columns: this CTA's half of O
+constexpr uint32_t kTmemS = 256;   // two 64-column S buffers
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
+
+static_assert(kOffKv % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "align");
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+struct Params {
+  Sm100Maps maps;
+  const int* block_table;
+  const int* seqlens;
+  const int* header;
+  const int* tile_prefix;
+  const int* split_base;
+  float* part_u;
+  float* part_lse;
+  __nv_bfloat16* u;
+  float* lse;
+  int* err;
+  int B, s_q, n_h, max_pages, page_size, num_pages;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+// Every lane of the warp polls; the warp agrees on the outcome.
+template <bool kCluster = false>
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err) {
+  const bool ok = mbar_wait<kCluster>(bar, parity, err, MLA_DEVFLAG_TIMEOUT);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    decode_sm100_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (sbase - raw_addr);
+  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cid = blockIdx.x >> 1;
+  const int chunk = cid / p.s_q, qrow = cid % p.s_q;
+  auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * i; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(KV_FULL + s), 1);
+      mbar_init(bar(KV_EMPTY + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(S_FULL + i), 1);
+      mbar_init(bar(S_EMPTY + i), 4);
+    }
+    mbar_init(bar(P_FULL), 4);
+    mbar_init(bar(PV_DONE), 1);
+    mbar_init(bar(X_FULL), 128);
+    mbar_init(bar(X_EMPTY), 128);
+    mbar_init(bar(Q_FULL), 1);
+    mbar_init(bar(Q_EMPTY), 1);
+    mbar_init(bar(MMA_FINAL), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpAlloc) {
+    tmem_alloc(sbase + kOffTmemSlot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    prefetch_tmap(&p.maps.q_lat);
+    prefetch_tmap(&p.maps.q_rope);
+    prefetch_tmap(&p.maps.kv_lat);
+    prefetch_tmap(&p.maps.kv_rope);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before anyone arrives on them
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base + kOffTmemSlot);
+  const int cs = p.header[1];
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      ChunkWalk walk;
+      walk.init(p.tile_prefix, p.B, chunk, cs);
+      Segment sg;
+      int g = 0, seg_i = 0, last_q = -1;
+      int last_n[kStages];
+      for (int s = 0; s < kStages; ++s) last_n[s] = -1;
+      bool ok = true;
+      while (ok && walk.next(sg)) {
+        if (seg_i > 0 && !(ok = mbar_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err, MLA_DEVFLAG_TIMEOUT)))
+          break;
+        const int qy = (sg.b * p.s_q + qrow) * p.n_h;
+        mbar_arrive_expect_tx(bar(Q_FULL), kQBytes);
+        for (int kb = 0; kb < 4; ++kb)
+          tma_load_2d(sbase + kOffQ + kb * kQBlk, &p.maps.q_lat, bar(Q_FULL),
+                      rank * kLatPerCta + kb * 64, qy);
+        tma_load_2d(sbase + kOffQ + 4 * kQBlk, &p.maps.q_rope, bar(Q_FULL),
+                    kDc + rank * kRopePerCta, qy);
+        last_q = seg_i;
+        const int* bt = p.block_table + (size_t)sg.b * p.max_pages;
+        for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+          const int s = g % kStages, n = g / kStages;
+          if (!(ok = mbar_wait(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT))) break;
+          const int tok = t * kTileTokens;
+          int page = bt[tok / p.page_size];
+          if (page < 0 || page >= p.num_pages) {
+            atomicOr(p.err, MLA_DEVFLAG_BAD_PAGE);
+            page = 0;
+          }
+          const int y = page * p.page_size + tok % p.page_size;
+          const uint32_t st = sbase + kOffKv + s * kStageBytes;
+          mbar_arrive_expect_tx(bar(KV_FULL + s), kStageBytes);
+          for (int kb = 0; kb < 4; ++kb)
+            tma_load_2d(st + kb * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
+                        rank * kLatPerCta + kb * 64, y);
+          tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(KV_FULL + s),
+                      kDc + rank * kRopePerCta, y);
+          last_n[s] = n;
+        }
+        ++seg_i;
+      }
+      // wait for this thread's own copies in flight before the CTA may exit
+      for (int s = 0; s < kStages; ++s)
+        if (last_n[s] >= 0) mbar_wait(bar(KV_FULL + s), last_n[s] & 1, p.err, MLA_DEVFLAG_TIMEOUT);
+      if (last_q >= 0) mbar_wait(bar(Q_FULL), last_q & 1, p.err, MLA_DEVFLAG_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdS = idesc_bf16(128, 64, false);
+    constexpr uint32_t kIdPV = idesc_bf16(128, kLatPerCta, true);
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.B, chunk, cs);
+    Segment sg;
+    int g = 0, seg_i = 0;
+    bool ok = true;
+    // O (+)= P . C for global tile gp; `first` = first tile of its segment
+    auto issue_pv = [&](int gp, bool first) -> bool {
+      if (!warp_wait(bar(P_FULL), gp & 1, p.err)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t st = sbase + kOffKv + (gp % kStages) * kStageBytes;
+        for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
+          const uint64_t a = smem_desc(sbase + kOffP + kk * 32, 16, 1024, kLayoutSW128);
+          const uint64_t b = smem_desc(st + kk * 2048, kKvBlk, 1024, kLayoutSW128);
+          umma_f16_ss(tmem + kTmemO, a, b, kIdPV, (first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(bar(KV_EMPTY + gp % kStages));
+        umma_commit(bar(PV_DONE));
+      }
+      __syncwarp();
+      return true;
+    };
+    while (ok && walk.next(sg)) {
+      if (!(ok = warp_wait(bar(Q_FULL), seg_i & 1, p.err))) break;
+      const int L = p.seqlens[sg.b];
+      const int n_t = sg.t1 - sg.t0;
+      for (int j = 0; j < n_t; ++j, ++g) {
+        const int t = sg.t0 + j, s = g % kStages;
+        if (!(ok = warp_wait(bar(KV_FULL + s), (g / kStages) & 1, p.err))) break;
+        const uint32_t st = sbase + kOffKv + s * kStageBytes;
+        const int rows_valid = L - t * kTileTokens;
+        if (rows_valid < kTileTokens) {
+          // rows past the sequence end may hold anything; make them zero so
+          // that 0-probability x garbage cannot turn into NaN in P . C
+          uint8_t* tile = base + kOffKv + s * kStageBytes;
+          for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
+            for (int kb = 0; kb < 4; ++kb)
+              if (lane < 8)
+                *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
+                    make_uint4(0, 0, 0, 0);
+            if (lane < 4)
+              *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (!(ok = warp_wait(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t dS = tmem + kTmemS + (g & 1) * 64;
+          uint32_t acc = 0;
+          for (int kb = 0; kb < 4; ++kb)
+            for (int ks = 0; ks < 4; ++ks) {  // 16 columns per MMA
+              const uint64_t a = smem_desc(sbase + kOffQ + kb * kQBlk + ks * 32, 16, 1024, kLayoutSW128);
+              const uint64_t b = smem_desc(st + kb * kKvBlk + ks * 32, 16, 1024, kLayoutSW128);
+              umma_f16_ss(dS, a, b, kIdS, acc);
+              acc = 1;
+            }
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t a = smem_desc(sbase + kOffQ + 4 * kQBlk + ks * 32, 16, 512, kLayoutSW64);
+            const uint64_t b = smem_desc(st + 4 * kKvBlk + ks * 32, 16, 512, kLayoutSW64);
+            umma_f16_ss(dS, a, b, kIdS, 1u);
+          }
+          umma_commit(bar(S_FULL + (g & 1)));
+          if (j == n_t - 1) umma_commit(bar(Q_EMPTY));
+        }
+        __syncwarp();
+        if (j > 0 && !(ok = issue_pv(g - 1, j == 1))) break;
+      }
+      if (!ok) break;
+      if (!(ok = issue_pv(g - 1, n_t == 1))) break;
+      ++seg_i;
+    }
+    // every MMA issued by this thread has completed before TMEM is freed
+    if (lane == 0) {
+      umma_commit(bar(MMA_FINAL));
+      mbar_wait(bar(MMA_FINAL), 0, p.err, MLA_DEVFLAG_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp >= kWarpSoftmax0) {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp - kWarpSoftmax0;
+    const int row = quad * 32 + lane;  // head
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t x_local = sbase + kOffX + row * 256;
+    const uint32_t x_remote = mapa(x_local, peer);
+    const uint32_t xfull_remote = mapa(bar(X_FULL), peer);
+    const uint32_t xempty_remote = mapa(bar(X_EMPTY), peer);
+    const uint32_t p_row = sbase + kOffP + row * 128;
+    const uint32_t sw = static_cast<uint32_t>(row & 7);
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.B, chunk, cs);
+    Segment sg;
+    int g = 0;
+    bool ok = true;
+    while (ok && walk.next(sg)) {
+      const int L = p.seqlens[sg.b];
+      const int L_eff = L - p.s_q + 1 + qrow;  // positions this query row may see
+      float m = -INFINITY, l = 0.f;
+      const int n_t = sg.t1 - sg.t0;
+      for (int j = 0; j < n_t; ++j, ++g) {
+        const int t = sg.t0 + j;
+        float s[64];
+        if (!(ok = warp_wait(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
+        tc_fence_after();
+        {
+          float (&s0)[32] = *reinterpret_cast<float(*)[32]>(&s[0]);
+          float (&s1)[32] = *reinterpret_cast<float(*)[32]>(&s[32]);
+          const uint32_t ta = tmem + lane_base + kTmemS + (g & 1) * 64;
+          tmem_ld32(ta, s0);
+          tmem_ld32(ta + 32, s1);
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(S_EMPTY + (g & 1)));
+
+        // exchange partial scores with the peer CTA
+        if (!(ok = warp_wait<true>(bar(X_EMPTY), (g & 1) ^ 1, p.err))) break;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          st_cluster_v4(x_remote + ((static_cast<uint32_t>(k) ^ sw) << 4), s[4 * k], s[4 * k + 1],
+                        s[4 * k + 2], s[4 * k + 3]);
+        mbar_arrive_remote(xfull_remote);
+        if (!(ok = warp_wait<true>(bar(X_FULL), g & 1, p.err))) break;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float4 v = ld_shared_v4(x_local + ((static_cast<uint32_t>(k) ^ sw) << 4));
+          s[4 * k] += v.x;
+          s[4 * k + 1] += v.y;
+          s[4 * k + 2] += v.z;
+          s[4 * k + 3] += v.w;
+        }
+        mbar_arrive_remote(xempty_remote);
+
+        // masked online softmax in log2 units
+        const int nv = L_eff - t * kTileTokens;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float x = c < nv ? s[c] * p.scale_log2 : -INFINITY;
+          s[c] = x;
+          mx = fmaxf(mx, x);
+        }
+        const float m_new = fmaxf(m, mx);
+        const bool resc = m_new > m + kRescaleThreshold;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = exp2f(m - m_new);
+          m = m_new;
+        }
+        const float m_use = m == -INFINITY ? 0.f : m;
+        float sum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(exp2f(s[c] - m_use), exp2f(s[c + 1] - m_use));
+          const float2 pf = __bfloat1622float2(pr);
+          sum += pf.x + pf.y;
+          pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        l = l * alpha + sum;
+
+        // the previous P . C must be done before P is overwritten or O rescaled
+        if (j > 0 && !(ok = warp_wait(bar(PV_DONE), (g - 1) & 1, p.err))) break;
+        tc_fence_after();
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          for (int c0 = 0; c0 < kLatPerCta; c0 += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + kTmemO + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tmem + lane_base + kTmemO + c0, o);
+          }
+          tmem_wait_st();
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(p_row + ((static_cast<uint32_t>(k) ^ sw) << 4), pk[4 * k], pk[4 * k + 1],
+                       pk[4 * k + 2], pk[4 * k + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(P_FULL));
+      }
+      if (!ok) break;
+
+      // epilogue: u = O / l (this CTA's 256 columns), lse in natural log
+      if (!(ok = warp_wait(bar(PV_DONE), (g - 1) & 1, p.err))) break;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const bool write = row < p.n_h;
+      const size_t orow = (size_t)(sg.b * p.s_q + qrow) * p.n_h + row;
+      const size_t slot = sg.whole ? 0 : (size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow;
+      for (int c0 = 0; c0 < kLatPerCta; c0 += 32) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + kTmemO + c0, o);
+        tmem_wait_ld();
+        if (!write) continue;
+        const int col = rank * kLatPerCta + c0;
+        if (sg.whole) {
+          uint4* dst = reinterpret_cast<uint4*>(p.u + orow * kDc + col);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 h2 =
+                  __floats2bfloat162_rn(o[8 * v + 2 * e] * inv, o[8 * v + 2 * e + 1] * inv);
+              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.part_u + (slot * p.n_h + row) * kDc + col);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
+                                 o[4 * v + 3] * inv);
+        }
+      }
+      if (write && rank == 0) {
+        if (sg.whole) {
+          if (p.lse != nullptr) p.lse[orow] = lse;
+        } else {
+          p.part_lse[slot * p.n_h + row] = lse;
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpAlloc) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
+}
+
+}  // namespace
+
+size_t decode_sm100_smem_bytes() { return kSmemBytes; }
+
+// Per device, once: opt in to the shared-memory size and count how many
+// 2-CTA clusters of this kernel can be resident at the same time.
+int decode_sm100_prepare() {
+  if (cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_sm100_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    n = sms / 2;
+  }
+  return n;
+}
+
+cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s) {
+  Params p;
+  p.maps = maps;
+  p.block_table = a.block_table;
+  p.seqlens = a.seqlens;
+  p.header = a.header;
+  p.tile_prefix = a.tile_prefix;
+  p.split_base = a.split_base;
+  p.part_u = a.part_u;
+  p.part_lse = a.part_lse;
+  p.u = static_cast<__nv_bfloat16*>(a.u);
+  p.lse = a.lse;
+  p.err = a.err;
+  p.B = a.B;
+  p.s_q = a.s_q;
+  p.n_h = a.n_h;
+  p.max_pages = a.max_pages;
+  p.page_size = a.page_size;
+  p.num_pages = a.num_pages;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  const dim3 grid(2 * a.num_chunks * a.s_q, 1, 1);
+  decode_sm100_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

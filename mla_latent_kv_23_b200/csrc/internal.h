@@ -1,0 +1,90 @@
+// Declarations shared by the translation units of libmla (not part of the ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "mla.h"
+
+namespace mla {
+
+constexpr int kTileTokens = 64;   // cache rows per attention tile
+constexpr int kMaxHeads = 128;    // query heads packed as the MMA M dimension
+
+// Workspace of mla_decode.  Header ints: [0] total tiles, [1] tiles per chunk,
+// [2] number of chunks, [3] split rows in use.
+struct WsLayout {
+  size_t header = 0, tile_prefix = 0, split_base = 0, part_lse = 0, part_u = 0, total = 0;
+  long long slots = 0;  // partial (u, lse) rows per head: (B + chunks) * s_q
+};
+WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks);
+
+// Everything a decode stage needs, resolved from mla_decode_params + workspace.
+struct DecodeArgs {
+  const void* q;
+  const void* kv;
+  const int* block_table;
+  const int* seqlens;
+  void* u;
+  float* lse;
+  int* header;
+  int* tile_prefix;
+  int* split_base;
+  float* part_u;
+  float* part_lse;
+  int* err;
+  int B, s_q, n_h, d_c, d_R, page_size, max_pages, num_pages, num_chunks;
+  float scale;
+  bool bf16;
+};
+
+cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s);
+
+// Tensor-core decode for n_h <= 128, d_c = 512, d_R = 64, bf16.
+// maps: q latent (box 64x128, SW128), q rope (32x128, SW64),
+//       kv latent (64x64, SW128), kv rope (32x64, SW64).
+struct Sm100Maps {
+  CUtensorMap q_lat, q_rope, kv_lat, kv_rope;
+};
+cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s);
+size_t decode_sm100_smem_bytes();
+
+// C[z][m][n] = sum_k A(z,m,k) * B(z,n,k), fp32 accumulation, generic strides
+// (element units), with a store epilogue that can
+//  - map the row through a paged block table (cache append),
+//  - split columns into segments of `seg` written `seg_stride` apart plus
+//    `col_off` (packed query / cache rows),
+//  - rotate consecutive column pairs by pos[m] * base^(-2k/seg) (RoPE).
+struct GemmArgs {
+  const void* A;
+  const void* Bm;
+  void* C;
+  int M, N, K, Z;
+  long long sAz, sAm, sAk;
+  long long sBz, sBn, sBk;
+  long long sCz, sCm;
+  int seg;               // column segment length (>= N means one segment)
+  long long seg_stride;  // distance between segments in C
+  long long col_off;     // added to every column
+  const int* pos;        // per-row position (RoPE and paged rows)
+  int rope;              // apply rotary pairs within each segment
+  double rope_base;
+  // paged rows: row of m = block_table[seq[m]*max_pages + pos[m]/page]*page + pos[m]%page
+  const int* seq;
+  const int* block_table;
+  int max_pages, page_size, num_pages;
+  int* err;
+  bool bf16;
+};
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// Per-head up-projection on the tensor cores (bf16).
+cudaError_t launch_up_proj_sm100(const void* u, const void* W_UV, void* o, int T, int n_h,
+                                 int d_c, int d_v, cudaStream_t s);
+
+}  // namespace mla

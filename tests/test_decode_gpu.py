@@ -1,0 +1,182 @@
+"""GPU parity of the whole path (absorb -> query -> decode -> up-projection)
+against the CPU oracle, at sizes the oracle finishes in seconds that still
+span many 64-token tiles, ragged tails, several KV chunks and both query-row
+counts, plus the edge cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_pipeline import (ATOL_REL, assert_parity, check_expanded, f64, run_pipeline, to_dev,
+                          to_dev_i32)
+from mla_latent_kv_23_b200 import mla, synth
+from oracle import mla_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+
+def v3_small(**kw):
+    base = dict(name="v3-small", B=3, s_q=1, n_h=128, d_model=512, d_c=512, d_h=128, d_v=128,
+                d_R=64, page_size=64, dtype="bf16", seqlens=(100, 1000, 777),
+                block_table="permuted", scale=1 / np.sqrt(192.0), seed=21)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+def some_heads(w, heads_first=None, heads_rest=(0, 1, 63, 64, 127)):
+    picks = []
+    for b in range(w.B):
+        hs = range(w.n_h) if (b == 0 and heads_first is None) else (heads_first if b == 0 else heads_rest)
+        for r in range(w.s_q):
+            for i in hs:
+                if i < w.n_h:
+                    picks.append((b, r, i))
+    return picks
+
+
+def test_tiny_config_full_pipeline():
+    w = synth.config("tiny")
+    inp = synth.draw(w)
+    out = run_pipeline(w, inp)
+    res = check_expanded(w, inp, out)
+    assert res["n"] == w.B * w.n_h
+    assert_parity(res)
+
+
+@pytest.mark.parametrize("s_q", [1, 2])
+@pytest.mark.parametrize("splits", [0, 1, 5])
+def test_v3_shape_ragged(s_q, splits):
+    w = v3_small(s_q=s_q)
+    inp = synth.draw(w)
+    out = run_pipeline(w, inp, num_splits=splits)
+    p = mla.decode_params(out["q"], out["cache"], out["bt"], out["seqlens"], out["u"], out["lse"],
+                          w.page_size, w.d_R, w.softmax_scale, splits)
+    tc, _ = mla.mla_decode_kernel_info(p)
+    assert tc == 1
+    assert_parity(check_expanded(w, inp, out, some_heads(w)))
+
+
+@pytest.mark.parametrize("s_q,seqlens", [(1, (1, 64, 65, 128, 129)), (2, (2, 64, 65, 130, 3))])
+def test_length_edges(s_q, seqlens):
+    w = v3_small(s_q=s_q, B=len(seqlens), seqlens=seqlens, block_table="identity")
+    inp = synth.draw(w)
+    out = run_pipeline(w, inp)
+    assert_parity(check_expanded(w, inp, out, some_heads(w, heads_first=(0, 5, 127))))
+
+
+def test_fewer_heads_and_bigger_pages():
+    w = v3_small(n_h=16, page_size=256, seqlens=(300, 513, 256))
+    inp = synth.draw(w)
+    out = run_pipeline(w, inp)
+    assert_parity(check_expanded(w, inp, out))
+
+
+def test_garbage_past_sequence_end_is_ignored():
+    w = v3_small(seqlens=(70, 200, 129), tail_fill="nan")
+    inp = synth.draw(w)
+    out = run_pipeline(w, inp)
+    assert torch.isfinite(out["u"].float()).all() and torch.isfinite(out["lse"]).all()
+    assert_parity(check_expanded(w, inp, out, some_heads(w, heads_first=(0, 77))))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_cuda_core_path_small_latent(dtype):
+    # d_c = 64, d_R = 16 goes to the CUDA-core kernel in either dtype
+    w = synth.config("tiny").with_(dtype=dtype, B=3, seqlens=(129, 129, 129), page_size=192,
+                                   block_table="permuted", full_pipeline=False)
+    inp = synth.draw(w)
+    out = run_pipeline(w, inp, num_splits=4)
+    res = check_expanded(w, inp, out)
+    assert_parity(res)
+
+
+def test_split_count_and_page_permutation_invariance():
+    w = v3_small(seqlens=(1500, 900, 2048), block_table="identity")
+    inp = synth.draw(w)
+    q = synth.random_q(w)
+    qd = to_dev(q, w)
+    cache = to_dev(inp["cache"], w)
+    bt = to_dev_i32(inp["block_table"])
+    sl = to_dev_i32(inp["seqlens"])
+    outs = {}
+    for splits in (1, 3, 16, 100):
+        outs[splits] = mla.decode(qd, cache, bt, sl, w.page_size, w.d_R, w.softmax_scale, splits)
+    u1, l1 = (f64(t) for t in outs[1])
+    for s, (u, l) in outs.items():
+        assert np.max(np.abs(f64(u) - u1) / (1 + np.abs(u1))) < ATOL_REL
+        assert np.max(np.abs(f64(l) - l1) / np.abs(l1)) < 1e-4
+    # same result bit for bit when the pages are moved and the table follows them
+    perm = np.random.default_rng(3).permutation(inp["num_pages"])
+    P = w.page_size
+    cache2 = np.empty_like(inp["cache"])
+    for p_old in range(inp["num_pages"]):
+        cache2[perm[p_old] * P:(perm[p_old] + 1) * P] = inp["cache"][p_old * P:(p_old + 1) * P]
+    bt2 = np.where(inp["block_table"] >= 0, perm[np.maximum(inp["block_table"], 0)], -1)
+    u2, l2 = mla.decode(qd, to_dev(cache2, w), to_dev_i32(bt2), sl, w.page_size, w.d_R,
+                        w.softmax_scale, 3)
+    assert torch.equal(u2, outs[3][0]) and torch.equal(l2, outs[3][1])
+    # and the decode matches the oracle's absorbed helper on the same query
+    ref = orc.decode_absorbed(q, inp["cache"], inp["block_table"], inp["seqlens"], w,
+                              [(b, 0, i) for b in range(w.B) for i in (0, 31, 127)])
+    for (b, r, i), (u_ref, lse_ref) in ref.items():
+        assert np.max(np.abs(u1[b, r, i] - u_ref) / (1 + np.abs(u_ref))) < ATOL_REL
+        assert abs(l1[b, r, i] - lse_ref) / abs(lse_ref) < 1e-3
+
+
+def test_row0_of_two_query_rows_equals_shorter_single_row():
+    w = v3_small(s_q=2, seqlens=(300, 64, 1025), block_table="identity")
+    inp = synth.draw(w)
+    q = to_dev(synth.random_q(w), w)
+    cache, bt = to_dev(inp["cache"], w), to_dev_i32(inp["block_table"])
+    u2, l2 = mla.decode(q, cache, bt, to_dev_i32(inp["seqlens"]), w.page_size, w.d_R,
+                        w.softmax_scale, 1)
+    u1, l1 = mla.decode(q[:, :1].contiguous(), cache, bt, to_dev_i32(inp["seqlens"] - 1),
+                        w.page_size, w.d_R, w.softmax_scale, 1)
+    assert torch.equal(u1[:, 0], u2[:, 0]) and torch.equal(l1[:, 0], l2[:, 0])
+
+
+def test_device_flags_for_bad_inputs():
+    w = v3_small(B=2, seqlens=(100, 200), block_table="identity")
+    inp = synth.draw(w)
+    q = to_dev(synth.random_q(w), w)
+    cache = to_dev(inp["cache"], w)
+    bt = inp["block_table"].copy()
+    bt[1, 1] = inp["num_pages"] + 5          # page id out of range
+    u, l = mla.decode(q, cache, to_dev_i32(bt), to_dev_i32(inp["seqlens"]), w.page_size, w.d_R,
+                      w.softmax_scale)
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_check_device_errors()
+    assert e.value.flags & mla.DEVFLAG_BAD_PAGE
+    sl = inp["seqlens"].copy()
+    sl[0] = 10 ** 6                          # longer than the block table allows
+    u, l = mla.decode(q, cache, to_dev_i32(inp["block_table"]), to_dev_i32(sl), w.page_size,
+                      w.d_R, w.softmax_scale)
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_check_device_errors()
+    assert e.value.flags & mla.DEVFLAG_BAD_SEQLEN
+    assert torch.all(u[0] == 0) and torch.all(torch.isneginf(l[0]))
+    assert mla.mla_check_device_errors() == 0   # flags were cleared
+
+
+def test_empty_batch():
+    q = torch.empty((0, 1, 128, 576), dtype=torch.bfloat16, device="cuda")
+    cache = torch.zeros((64, 576), dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros((0, 1), dtype=torch.int32, device="cuda")
+    sl = torch.zeros((0,), dtype=torch.int32, device="cuda")
+    u, l = mla.decode(q, cache, bt, sl, 64, 64, 0.07)
+    assert u.shape == (0, 1, 128, 512)
+
+
+def test_absorb_and_query_against_oracle():
+    w = v3_small(B=2, d_model=384, s_q=2, seqlens=(5000, 7))
+    inp = synth.draw(w)
+    from gpu_pipeline import absorb_and_query
+    q, W_QK = absorb_and_query(w, inp)
+    wqk_ref = orc.absorb_weights(inp["W_UK"], inp["W_Q"])
+    e = np.abs(f64(W_QK) - wqk_ref) / (1e-2 + np.abs(wqk_ref))
+    assert e.max() < 1e-2   # bf16 output rounding (2^-9) of an fp32-accumulated sum
+    qd = f64(q)
+    for b in range(w.B):
+        for r in range(w.s_q):
+            for i in (0, 100):
+                qref = orc.absorbed_query(inp, w, b, r, i)
+                assert np.max(np.abs(qd[b, r, i] - qref) / (1 + np.abs(qref))) < 2e-2
