@@ -30,12 +30,24 @@ TILE_TOKENS = 64  # cache rows per decode tile
 # ----------------------------------------------------------------------------
 # storage-type rounding
 # ----------------------------------------------------------------------------
-def bf16_round(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bf16 (ties to even); float32 out."""
+def bf16_round(x: np.ndarray, inplace: bool = False) -> np.ndarray:
+    """Round float32 values to the nearest bf16 (ties to even); float32 out.
+
+    Works on the bit pattern in uint32 arithmetic (finite values, infinities
+    and the NaNs drawn here never carry out of 32 bits), in chunks to bound
+    temporaries."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    b = x.view(np.uint32).astype(np.uint64)
-    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
-    return b.astype(np.uint32).view(np.float32).reshape(x.shape)
+    if not inplace:
+        x = x.copy()
+    b = x.reshape(-1).view(np.uint32)
+    step = 1 << 24
+    for i in range(0, b.size, step):
+        c = b[i:i + step]
+        lsb = (c >> 16) & 1
+        c += np.uint32(0x7FFF)
+        c += lsb
+        c &= np.uint32(0xFFFF0000)
+    return x
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -117,19 +129,44 @@ _TAGS = {"seqlens": 1, "perm": 2, "cache": 3, "outlier": 4, "h_q": 5, "W_Q": 6,
          "W_QR": 7, "W_UK": 8, "W_UV": 9, "W_DKV": 10, "W_KR": 11, "h_ctx": 12, "tail": 13}
 
 
-def _rng(seed: int, tag: str) -> np.random.Generator:
-    return np.random.default_rng([int(seed), _TAGS[tag]])
+_BLOCK = 1 << 22  # elements per independently seeded block of a large tensor
 
 
-def _normal(seed: int, tag: str, shape, std: float = 1.0) -> np.ndarray:
-    x = _rng(seed, tag).standard_normal(size=shape, dtype=np.float32)
+def _rng(seed: int, tag: str, block: int = -1) -> np.random.Generator:
+    key = [int(seed), _TAGS[tag]] + ([] if block < 0 else [int(block)])
+    return np.random.default_rng(key)
+
+
+def _fill_block(flat, k, seed, tag, std, dtype):
+    view = flat[k * _BLOCK:(k + 1) * _BLOCK]
+    _rng(seed, tag, k).standard_normal(out=view, dtype=np.float32)
     if std != 1.0:
-        x *= np.float32(std)
-    return x
+        view *= np.float32(std)
+    if dtype == "bf16":
+        bf16_round(view, inplace=True)
+
+
+def _normal(seed: int, tag: str, shape, std: float = 1.0, dtype: str = "fp32") -> np.ndarray:
+    """N(0, std^2) draws, rounded to `dtype`.  Block k of the flattened tensor
+    comes from stream default_rng([seed, tag, k]), so the values do not depend
+    on how many threads fill the blocks."""
+    out = np.empty(shape, dtype=np.float32)
+    flat = out.reshape(-1)
+    nblk = (flat.size + _BLOCK - 1) // _BLOCK
+    if nblk <= 1:
+        for k in range(nblk):
+            _fill_block(flat, k, seed, tag, std, dtype)
+        return out
+    import concurrent.futures as cf
+    import os
+    with cf.ThreadPoolExecutor(max_workers=min(nblk, os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda k: _fill_block(flat, k, seed, tag, std, dtype), range(nblk)))
+    return out
 
 
 def _store(x: np.ndarray, dtype: str) -> np.ndarray:
-    return bf16_round(x) if dtype == "bf16" else np.ascontiguousarray(x, dtype=np.float32)
+    """Round an array drawn in float32 to the storage type (in place)."""
+    return bf16_round(x, inplace=True) if dtype == "bf16" else np.ascontiguousarray(x, dtype=np.float32)
 
 
 def draw_seqlens(w: Workload) -> np.ndarray:
@@ -197,13 +234,14 @@ def draw(w: Workload, with_weights: bool = True) -> dict:
     if w.full_pipeline:
         assert w.seqlens is not None and len(set(w.seqlens)) == 1
         L = int(w.seqlens[0])
-        out["h_ctx"] = _store(_normal(w.seed, "h_ctx", (w.B, L, w.d_model)), dt)
-        out["W_DKV"] = _store(_normal(w.seed, "W_DKV", (w.d_c, w.d_model), 1 / math.sqrt(w.d_model)), dt)
-        out["W_KR"] = _store(_normal(w.seed, "W_KR", (w.d_R, w.d_model), 1 / math.sqrt(w.d_model)), dt)
+        out["h_ctx"] = _normal(w.seed, "h_ctx", (w.B, L, w.d_model), 1.0, dt)
+        out["W_DKV"] = _normal(w.seed, "W_DKV", (w.d_c, w.d_model), 1 / math.sqrt(w.d_model), dt)
+        out["W_KR"] = _normal(w.seed, "W_KR", (w.d_R, w.d_model), 1 / math.sqrt(w.d_model), dt)
         # the query tokens are the last s_q tokens appended to the context
         out["h_q"] = np.ascontiguousarray(out["h_ctx"][:, L - w.s_q:, :])
     else:
-        cache = _normal(w.seed, "cache", (rows, w.width))
+        plain = w.outlier_frac == 0 and w.tail_fill == "random"
+        cache = _normal(w.seed, "cache", (rows, w.width), 1.0, dt if plain else "fp32")
         if w.outlier_frac > 0:
             valid = np.concatenate([cache_row_ids(w, bt, b, int(seqlens[b])) for b in range(w.B)])
             k = max(1, int(round(w.outlier_frac * valid.size)))
@@ -214,24 +252,26 @@ def draw(w: Workload, with_weights: bool = True) -> dict:
             for b in range(w.B):
                 used[cache_row_ids(w, bt, b, int(seqlens[b]))] = True
             cache[~used] = np.nan if w.tail_fill == "nan" else 0.0
-        out["cache"] = _store(cache, dt)
+        out["cache"] = cache if plain else _store(cache, dt)
         if with_weights:
-            out["h_q"] = _store(_normal(w.seed, "h_q", (w.B, w.s_q, w.d_model)), dt)
+            out["h_q"] = _normal(w.seed, "h_q", (w.B, w.s_q, w.d_model), 1.0, dt)
     if with_weights:
         fi = 1 / math.sqrt(w.d_model)
-        out["W_Q"] = _store(_normal(w.seed, "W_Q", (w.n_h, w.d_h, w.d_model), fi), dt)
-        out["W_QR"] = _store(_normal(w.seed, "W_QR", (w.n_h, w.d_R, w.d_model), fi), dt)
-        out["W_UK"] = _store(_normal(w.seed, "W_UK", (w.n_h, w.d_h, w.d_c), 1 / math.sqrt(w.d_c)), dt)
-        out["W_UV"] = _store(_normal(w.seed, "W_UV", (w.n_h, w.d_v, w.d_c), 1 / math.sqrt(w.d_c)), dt)
+        out["W_Q"] = _normal(w.seed, "W_Q", (w.n_h, w.d_h, w.d_model), fi, dt)
+        out["W_QR"] = _normal(w.seed, "W_QR", (w.n_h, w.d_R, w.d_model), fi, dt)
+        out["W_UK"] = _normal(w.seed, "W_UK", (w.n_h, w.d_h, w.d_c), 1 / math.sqrt(w.d_c), dt)
+        out["W_UV"] = _normal(w.seed, "W_UV", (w.n_h, w.d_v, w.d_c), 1 / math.sqrt(w.d_c), dt)
     return out
 
 
 def random_q(w: Workload, seed_tag: int = 0) -> np.ndarray:
     """An absorbed query tensor [B, s_q, n_h, d_c + d_R] drawn directly.
 
-    Used only where a test needs decode inputs without the query projections
-    (latent part N(0, 0.25), RoPE part N(0, 1), the spreads the V3 projections
-    give); parity against the expanded oracle always forms q from h instead.
+    Used where the decode is judged on its own bf16 inputs rather than
+    through query formation: the long-context stress workload and the
+    invariance checks.  The latent part is N(0, 0.25) and the RoPE part
+    N(0, 1), the spreads the V3-shaped projections of N(0, 1) hidden states
+    give.
     """
     g = np.random.default_rng([w.seed, 100 + seed_tag])
     q = g.standard_normal(size=(w.B, w.s_q, w.n_h, w.width), dtype=np.float32)

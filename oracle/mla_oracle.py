@@ -206,10 +206,15 @@ def absorbed_query(inp: dict, w, b: int, r: int, i: int, W_QK_i=None) -> np.ndar
     return np.concatenate([qlat, qr])
 
 
-def decode_absorbed(q: np.ndarray, cache, block_table, seqlens, w, picks=None):
+def decode_absorbed(q: np.ndarray, cache, block_table, seqlens, w, picks=None,
+                    with_abs: bool = False, W_UV=None):
     """Absorbed decode from an explicit query tensor q [B, s_q, n_h, d_c + d_R]:
     s_j = q^lat.c_j + q^R.k^R_j, a = softmax(scale s) over j <= L - s_q + r,
-    u = sum_j a_j c_j.  Returns dict (b, r, i) -> (u [d_c], lse)."""
+    u = sum_j a_j c_j.  Returns dict (b, r, i) -> (u [d_c], lse).
+
+    with_abs: the value is a dict with u, lse and abs_c = sum_j a_j |c_j|
+    (the scale against which rounding of the weights a_j is measured); given
+    W_UV as well, also o = W^UV_i u and abs_v = sum_j a_j |W^UV_i c_j|."""
     if picks is None:
         picks = [(b, r, i) for b in range(w.B) for r in range(w.s_q) for i in range(w.n_h)]
     by_seq = {}
@@ -226,7 +231,19 @@ def decode_absorbed(q: np.ndarray, cache, block_table, seqlens, w, picks=None):
             m = s.max()
             e = np.exp(s - m)
             z = e.sum()
-            out[(b, r, i)] = ((e / z) @ rows[:n_valid, :w.d_c], m + math.log(z))
+            a = e / z
+            C = rows[:n_valid, :w.d_c]
+            u = a @ C
+            lse = m + math.log(z)
+            if not with_abs:
+                out[(b, r, i)] = (u, lse)
+                continue
+            d = dict(u=u, lse=lse, abs_c=a @ np.abs(C))
+            if W_UV is not None:
+                Wi = np.asarray(W_UV[i], f64)
+                d["o"] = Wi @ u
+                d["abs_v"] = a @ np.abs(C @ Wi.T)
+            out[(b, r, i)] = d
     return out
 
 

@@ -103,6 +103,59 @@ def check_expanded(w, inp, out, picks=None):
     return dict(o=worst_o, lse=worst_lse, u=worst_u, n=len(ref))
 
 
+# Tighter bounds for decode-only comparisons on identical bf16 inputs, derived
+# from the kernel's arithmetic: each softmax weight is rounded to bf16 before
+# the P.C contraction (relative error <= 2^-9, normalised by the sum of the
+# rounded weights), u is stored in bf16 (relative error <= 2^-9), and the
+# up-projection reads that bf16 u and stores o in bf16; scores, exponentials
+# and every accumulation are fp32.  So, up to fp32 terms,
+#   |du_k| <= 2^-8 sum_j a_j |c_jk| + 2^-9 |u_k|
+#   |do_k| <= 2^-8 sum_j a_j |(W c_j)_k| + 2^-9 sum_c |W_kc| |u_c| + 2^-9 |o_k|
+# (a weight error moves a whole cached row, so it reaches o through W^UV).
+# The checks allow 2x these.
+def tight_u_bound(u_ref, abs_c):
+    return 2.0 * (2.0 ** -8 * abs_c + 2.0 ** -9 * np.abs(u_ref)) + 1e-6
+
+
+def tight_o_bound(o_ref, abs_v, W_i, u_ref):
+    return 2.0 * (2.0 ** -8 * abs_v + 2.0 ** -9 * (np.abs(W_i) @ np.abs(u_ref)) +
+                  2.0 ** -9 * np.abs(o_ref)) + 1e-6
+
+
+def check_absorbed(w, q, inp, out, picks, W_UV=None):
+    """u / lse / o of a decode run on the generator's q against the oracle's
+    absorbed helper (itself pinned to the expanded definition)."""
+    ref = orc.decode_absorbed(q, inp["cache"], inp["block_table"], inp["seqlens"], w, picks,
+                              with_abs=True, W_UV=W_UV)
+    u, lse = f64(out["u"]), f64(out["lse"])
+    o = f64(out["o"]) if out.get("o") is not None else None
+    res = dict(o=0.0, u=0.0, lse=0.0, tight=0.0, tight_o=0.0, n=len(ref))
+    for (b, r, i), d in ref.items():
+        u_ref, lse_ref = d["u"], d["lse"]
+        res["u"] = max(res["u"], float(np.max(np.abs(u[b, r, i] - u_ref) / (1 + np.abs(u_ref)))))
+        res["tight"] = max(res["tight"], float(np.max(np.abs(u[b, r, i] - u_ref) /
+                                                      tight_u_bound(u_ref, d["abs_c"]))))
+        res["lse"] = max(res["lse"], abs(lse[b, r, i] - lse_ref) / abs(lse_ref))
+        if o is not None and W_UV is not None:
+            o_ref = d["o"]
+            err = np.abs(o[b, r, i] - o_ref)
+            res["o"] = max(res["o"], float(np.max(err / (1 + np.abs(o_ref)))))
+            bound = tight_o_bound(o_ref, d["abs_v"], np.asarray(W_UV[i], np.float64), u_ref)
+            res["tight_o"] = max(res["tight_o"], float(np.max(err / bound)))
+    return res
+
+
+def assert_tight(res, o_north_star=True):
+    """Tight bounds on u (and o when present); the benchmark spec's tolerance on
+    u and lse always, and on o unless o_north_star is False."""
+    assert res["u"] <= ATOL_REL, res
+    assert res["lse"] <= LSE_REL, res
+    if o_north_star:
+        assert res["o"] <= ATOL_REL, res
+    assert res["tight"] <= 1.0, res
+    assert res["tight_o"] <= 1.0, res
+
+
 def assert_parity(res):
     assert res["o"] <= ATOL_REL, res
     assert res["u"] <= ATOL_REL, res
