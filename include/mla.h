@@ -179,6 +179,11 @@ mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_c
  *   u     [T, n_h, d_c]   device, read   (T = B * s_q)
  *   W_UV  [n_h, d_v, d_c] device, read
  *   o     [T, n_h, d_v]   device, written
+ * The bf16 tensor-core kernel (d_v = 128, d_c a multiple of 64 up to 512)
+ * starts reading W_UV before the previous kernel on the stream has finished
+ * (programmatic dependent launch; u is read only after it has).  So W_UV
+ * must not be written by the kernel launched immediately before this call
+ * on the same stream; weights written earlier, or by a copy, are fine.
  */
 mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c,
                        int d_v, mla_dtype dtype, void* stream);

@@ -29,6 +29,7 @@ struct DeviceInfo {
   int sm_count = 0;
   int cc_major = 0, cc_minor = 0;
   int max_clusters = 0;  // co-resident 2-CTA clusters of the tensor-core kernel
+  bool up_proj_tc = false;
   int* flags = nullptr;  // device address of g_device_flags
 };
 
@@ -64,6 +65,7 @@ mla_status device_info(const DeviceInfo** out) {
     if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.flags), g_device_flags)) != cudaSuccess)
       return cuda_status(e);
     d.max_clusters = (d.cc_major == 10) ? decode_sm100_prepare() : 0;
+    d.up_proj_tc = (d.cc_major == 10) && up_proj_sm100_prepare() != 0;
     if (g_encode == nullptr) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -431,6 +433,23 @@ mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h,
   const DeviceInfo* d = nullptr;
   mla_status st = device_info(&d);
   if (st != MLA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->up_proj_tc && g_encode != nullptr && dtype == MLA_DTYPE_BF16 && d_v == 128 &&
+      d_c % 64 == 0 && d_c <= 512) {
+    CUtensorMap w_map, u_map;
+    if ((st = encode_2d(&w_map, W_UV, d_c, (uint64_t)n_h * d_v, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return st;
+    const cuuint64_t dims[3] = {(cuuint64_t)d_c, (cuuint64_t)n_h, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)d_c * 2, (cuuint64_t)n_h * d_c * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)up_proj_sm100_box_rows(T)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (g_encode(&u_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(u), dims, strides,
+                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+    return cuda_status(launch_up_proj_sm100(w_map, u_map, o, d->flags, T, n_h, d_c, s));
+  }
   GemmArgs g = {};
   g.A = u;     // A(z = head, m = t, k = c) = u[t][z][c]
   g.Bm = W_UV; // B(z, n = v, k = c) = W_UV[z][v][c]
@@ -450,7 +469,7 @@ mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h,
   g.seg = INT_MAX;
   g.err = d->flags;
   g.bf16 = dtype == MLA_DTYPE_BF16;
-  return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_gemm(g, s));
 }
 
 mla_status mla_check_device_errors(void* stream, int* flags) {

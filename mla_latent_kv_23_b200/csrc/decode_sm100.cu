@@ -17,16 +17,23 @@
 // columns, and the two partial S tiles are exchanged through distributed
 // shared memory.  Both CTAs then hold the same S (fp32 addition commutes),
 // make bit-identical softmax decisions, and each accumulates its own half of
-// O = P . C (N = 256).  TMEM per CTA: O 256 columns + 2 S buffers of 64.
+// O = P . C (N = 256).  TMEM per CTA: O 256 columns, two 64-column S
+// buffers, two 32-column P buffers (bf16 pairs; P is the A operand of P . C
+// straight from TMEM).
 //
 // One shared-memory tile serves both contractions: a TMA load with 128-byte
 // swizzle writes each 64-column block as 64 rows x 128 B, which is the
 // K-major operand layout of S = Q K^T and the MN-major operand layout of
 // O = P C at the same time.
 //
-// Warp roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and
-// zeroes cache rows past the end of a sequence), warp 2 = TMEM allocator,
-// warps 4-7 = softmax / correction / epilogue, one thread per head (TMEM lane).
+// Pipeline.  Three tile stages.  The MMA thread issues S two tiles ahead of
+// P . C (S_{j+2} after PV_j), so a P . C never waits on a load that has just
+// started, and a stage is refilled as soon as its P . C retires.
+//
+// Warp roles (256 threads): warp 0 = TMA producer (the whole warp prefetches
+// block-table entries, lane 0 issues copies), warp 1 = MMA issuer (and zeroes
+// cache rows past the end of a sequence), warp 2 = TMEM allocator, warps 4-7
+// = softmax / correction / epilogue, one thread per head (TMEM lane).
 //
 // Work: the plan stage cuts the batch's tiles into equal chunks; cluster c
 // handles chunk c / s_q for query row c % s_q, walking its segments in order.
@@ -43,7 +50,7 @@ using namespace ptx;
 
 constexpr int kThreads = 256;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpAlloc = 2, kWarpSoftmax0 = 4;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kDc = 512;
 constexpr int kLatPerCta = 256, kRopePerCta = 32;
 
@@ -53,23 +60,21 @@ constexpr uint32_t kQBytes = 4 * kQBlk + kQRope;         // 73728
 constexpr uint32_t kKvBlk = 64 * 128;                    // tile: 64 rows x 64 cols, SW128
 constexpr uint32_t kKvRope = 64 * 64;                    // tile: 64 rows x 32 cols, SW64
 constexpr uint32_t kStageBytes = 4 * kKvBlk + kKvRope;   // 36864
-constexpr uint32_t kPBytes = 128 * 128;                  // P: 128 rows x 64 tokens bf16, SW128
 constexpr uint32_t kXBytes = 128 * 256;                  // peer partial S: 128 x 64 fp32
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKv = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;
-constexpr uint32_t kOffX = kOffP + kPBytes;
+constexpr uint32_t kOffX = kOffKv + kStages * kStageBytes;
 constexpr uint32_t kOffBar = kOffX + kXBytes;
 
 enum Bar {
   KV_FULL = 0,
   KV_EMPTY = KV_FULL + kStages,
-  S_FULL = KV_EMPTY + kStages,
-  S_EMPTY = S_FULL + 2,
-  P_FULL = S_EMPTY + 2,
-  PV_DONE,
-  X_FULL,
+  S_FULL = KV_EMPTY + kStages,   // [2]
+  S_EMPTY = S_FULL + 2,          // [2]
+  P_FULL = S_EMPTY + 2,          // [2] per P buffer
+  PV_DONE = P_FULL + 2,          // [2] per P buffer
+  X_FULL = PV_DONE + 2,
   X_EMPTY,
   Q_FULL,
   Q_EMPTY,
@@ -83,9 +88,10 @@ constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;     // 256 columns: this CTA's half of O
 constexpr uint32_t kTmemS = 256;   // two 64-column S buffers
+constexpr uint32_t kTmemP = 384;   // two 32-column P buffers (64 bf16 per row each)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
-static_assert(kOffKv % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "align");
+static_assert(kOffKv % 1024 == 0 && kStageBytes % 1024 == 0 && kOffX % 1024 == 0, "align");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct Params {
@@ -131,9 +137,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(S_FULL + i), 1);
       mbar_init(bar(S_EMPTY + i), 4);
+      mbar_init(bar(P_FULL + i), 4);
+      mbar_init(bar(PV_DONE + i), 1);
     }
-    mbar_init(bar(P_FULL), 4);
-    mbar_init(bar(PV_DONE), 1);
     mbar_init(bar(X_FULL), 128);
     mbar_init(bar(X_EMPTY), 128);
     mbar_init(bar(Q_FULL), 1);
@@ -156,52 +162,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // the peer's barriers exist before anyone arrives on them
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base + kOffTmemSlot);
+  // everything above overlaps the plan kernel; its results are read below
+  pdl_wait_previous();
+  pdl_launch_dependents();
   const int cs = p.header[1];
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      ChunkWalk walk;
-      walk.init(p.tile_prefix, p.B, chunk, cs);
-      Segment sg;
-      int g = 0, seg_i = 0, last_q = -1;
-      int last_n[kStages];
-      for (int s = 0; s < kStages; ++s) last_n[s] = -1;
-      bool ok = true;
-      while (ok && walk.next(sg)) {
-        if (seg_i > 0 && !(ok = mbar_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err, MLA_DEVFLAG_TIMEOUT)))
-          break;
-        const int qy = (sg.b * p.s_q + qrow) * p.n_h;
-        mbar_arrive_expect_tx(bar(Q_FULL), kQBytes);
-        for (int kb = 0; kb < 4; ++kb)
-          tma_load_2d(sbase + kOffQ + kb * kQBlk, &p.maps.q_lat, bar(Q_FULL),
-                      rank * kLatPerCta + kb * 64, qy);
-        tma_load_2d(sbase + kOffQ + 4 * kQBlk, &p.maps.q_rope, bar(Q_FULL),
-                    kDc + rank * kRopePerCta, qy);
-        last_q = seg_i;
-        const int* bt = p.block_table + (size_t)sg.b * p.max_pages;
-        for (int t = sg.t0; t < sg.t1; ++t, ++g) {
-          const int s = g % kStages, n = g / kStages;
-          if (!(ok = mbar_wait(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT))) break;
-          const int tok = t * kTileTokens;
-          int page = bt[tok / p.page_size];
-          if (page < 0 || page >= p.num_pages) {
-            atomicOr(p.err, MLA_DEVFLAG_BAD_PAGE);
-            page = 0;
-          }
-          const int y = page * p.page_size + tok % p.page_size;
-          const uint32_t st = sbase + kOffKv + s * kStageBytes;
-          mbar_arrive_expect_tx(bar(KV_FULL + s), kStageBytes);
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.B, chunk, cs);
+    Segment sg;
+    int g = 0, seg_i = 0, last_q = -1;
+    int last_n[kStages];
+    for (int s = 0; s < kStages; ++s) last_n[s] = -1;
+    bool ok = true;
+    while (ok && walk.next(sg)) {
+      if (lane == 0) {
+        if (seg_i > 0) ok = mbar_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err, MLA_DEVFLAG_TIMEOUT);
+        if (ok) {
+          const int qy = (sg.b * p.s_q + qrow) * p.n_h;
+          mbar_arrive_expect_tx(bar(Q_FULL), kQBytes);
           for (int kb = 0; kb < 4; ++kb)
-            tma_load_2d(st + kb * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
-                        rank * kLatPerCta + kb * 64, y);
-          tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(KV_FULL + s),
-                      kDc + rank * kRopePerCta, y);
-          last_n[s] = n;
+            tma_load_2d(sbase + kOffQ + kb * kQBlk, &p.maps.q_lat, bar(Q_FULL),
+                        rank * kLatPerCta + kb * 64, qy);
+          tma_load_2d(sbase + kOffQ + 4 * kQBlk, &p.maps.q_rope, bar(Q_FULL),
+                      kDc + rank * kRopePerCta, qy);
+          last_q = seg_i;
         }
-        ++seg_i;
       }
-      // wait for this thread's own copies in flight before the CTA may exit
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int* bt = p.block_table + (size_t)sg.b * p.max_pages;
+      for (int t0 = sg.t0; ok && t0 < sg.t1; t0 += 32) {
+        // each lane fetches the page of one upcoming tile
+        int my_page = 0;
+        if (t0 + lane < sg.t1) {
+          my_page = bt[((t0 + lane) * kTileTokens) / p.page_size];
+          if (my_page < 0 || my_page >= p.num_pages) {
+            atomicOr(p.err, MLA_DEVFLAG_BAD_PAGE);
+            my_page = 0;
+          }
+        }
+        const int n_here = min(32, sg.t1 - t0);
+        for (int i = 0; i < n_here; ++i, ++g) {
+          const int page = __shfl_sync(0xffffffffu, my_page, i);
+          if (lane == 0) {
+            const int s = g % kStages, n = g / kStages;
+            ok = mbar_wait(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT);
+            if (ok) {
+              const int tok = (t0 + i) * kTileTokens;
+              const int y = page * p.page_size + tok % p.page_size;
+              const uint32_t st = sbase + kOffKv + s * kStageBytes;
+              mbar_arrive_expect_tx(bar(KV_FULL + s), kStageBytes);
+              for (int kb = 0; kb < 4; ++kb)
+                tma_load_2d(st + kb * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
+                            rank * kLatPerCta + kb * 64, y);
+              tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(KV_FULL + s),
+                          kDc + rank * kRopePerCta, y);
+              last_n[s] = n;
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+        }
+      }
+      ++seg_i;
+    }
+    // wait for this thread's own copies in flight before the CTA may exit
+    if (lane == 0) {
       for (int s = 0; s < kStages; ++s)
         if (last_n[s] >= 0) mbar_wait(bar(KV_FULL + s), last_n[s] & 1, p.err, MLA_DEVFLAG_TIMEOUT);
       if (last_q >= 0) mbar_wait(bar(Q_FULL), last_q & 1, p.err, MLA_DEVFLAG_TIMEOUT);
@@ -214,21 +241,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ChunkWalk walk;
     walk.init(p.tile_prefix, p.B, chunk, cs);
     Segment sg;
-    int g = 0, seg_i = 0;
+    int g0 = 0, seg_i = 0;
     bool ok = true;
-    // O (+)= P . C for global tile gp; `first` = first tile of its segment
-    auto issue_pv = [&](int gp, bool first) -> bool {
-      if (!warp_wait(bar(P_FULL), gp & 1, p.err)) return false;
+    // S = Q . tile^T for global tile g (tile index t of the segment's sequence)
+    auto issue_s = [&](int g, int t, int L, bool last) -> bool {
+      const int s = g % kStages;
+      if (!warp_wait(bar(KV_FULL + s), (g / kStages) & 1, p.err)) return false;
+      const int rows_valid = L - t * kTileTokens;
+      if (rows_valid < kTileTokens) {
+        // rows past the sequence end may hold anything; make them zero so
+        // that 0-probability x garbage cannot turn into NaN in P . C
+        uint8_t* tile = base + kOffKv + s * kStageBytes;
+        for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
+          if (lane < 8)
+            for (int kb = 0; kb < 4; ++kb)
+              *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
+                  make_uint4(0, 0, 0, 0);
+          if (lane < 4)
+            *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (!warp_wait(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t st = sbase + kOffKv + (gp % kStages) * kStageBytes;
-        for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
-          const uint64_t a = smem_desc(sbase + kOffP + kk * 32, 16, 1024, kLayoutSW128);
-          const uint64_t b = smem_desc(st + kk * 2048, kKvBlk, 1024, kLayoutSW128);
-          umma_f16_ss(tmem + kTmemO, a, b, kIdPV, (first && kk == 0) ? 0u : 1u);
+        const uint32_t st = sbase + kOffKv + s * kStageBytes;
+        const uint32_t dS = tmem + kTmemS + (g & 1) * 64;
+        uint32_t acc = 0;
+        for (int kb = 0; kb < 4; ++kb)
+          for (int ks = 0; ks < 4; ++ks) {  // 16 columns per MMA
+            const uint64_t a = smem_desc(sbase + kOffQ + kb * kQBlk + ks * 32, 16, 1024, kLayoutSW128);
+            const uint64_t b = smem_desc(st + kb * kKvBlk + ks * 32, 16, 1024, kLayoutSW128);
+            umma_f16_ss(dS, a, b, kIdS, acc);
+            acc = 1;
+          }
+        for (int ks = 0; ks < 2; ++ks) {
+          const uint64_t a = smem_desc(sbase + kOffQ + 4 * kQBlk + ks * 32, 16, 512, kLayoutSW64);
+          const uint64_t b = smem_desc(st + 4 * kKvBlk + ks * 32, 16, 512, kLayoutSW64);
+          umma_f16_ss(dS, a, b, kIdS, 1u);
         }
-        umma_commit(bar(KV_EMPTY + gp % kStages));
-        umma_commit(bar(PV_DONE));
+        umma_commit(bar(S_FULL + (g & 1)));
+        if (last) umma_commit(bar(Q_EMPTY));
+      }
+      __syncwarp();
+      return true;
+    };
+    // O (+)= P . C for global tile g; `first` = first tile of its segment
+    auto issue_pv = [&](int g, bool first) -> bool {
+      if (!warp_wait(bar(P_FULL + (g & 1)), (g >> 1) & 1, p.err)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t st = sbase + kOffKv + (g % kStages) * kStageBytes;
+        const uint32_t pa = tmem + kTmemP + (g & 1) * 32;
+        for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
+          const uint64_t b = smem_desc(st + kk * 2048, kKvBlk, 1024, kLayoutSW128);
+          umma_f16_ts(tmem + kTmemO, pa + kk * 8, b, kIdPV, (first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(bar(KV_EMPTY + g % kStages));
+        umma_commit(bar(PV_DONE + (g & 1)));
       }
       __syncwarp();
       return true;
@@ -237,52 +309,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!(ok = warp_wait(bar(Q_FULL), seg_i & 1, p.err))) break;
       const int L = p.seqlens[sg.b];
       const int n_t = sg.t1 - sg.t0;
-      for (int j = 0; j < n_t; ++j, ++g) {
-        const int t = sg.t0 + j, s = g % kStages;
-        if (!(ok = warp_wait(bar(KV_FULL + s), (g / kStages) & 1, p.err))) break;
-        const uint32_t st = sbase + kOffKv + s * kStageBytes;
-        const int rows_valid = L - t * kTileTokens;
-        if (rows_valid < kTileTokens) {
-          // rows past the sequence end may hold anything; make them zero so
-          // that 0-probability x garbage cannot turn into NaN in P . C
-          uint8_t* tile = base + kOffKv + s * kStageBytes;
-          for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
-            for (int kb = 0; kb < 4; ++kb)
-              if (lane < 8)
-                *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
-                    make_uint4(0, 0, 0, 0);
-            if (lane < 4)
-              *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
-                  make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
-        if (!(ok = warp_wait(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err))) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t dS = tmem + kTmemS + (g & 1) * 64;
-          uint32_t acc = 0;
-          for (int kb = 0; kb < 4; ++kb)
-            for (int ks = 0; ks < 4; ++ks) {  // 16 columns per MMA
-              const uint64_t a = smem_desc(sbase + kOffQ + kb * kQBlk + ks * 32, 16, 1024, kLayoutSW128);
-              const uint64_t b = smem_desc(st + kb * kKvBlk + ks * 32, 16, 1024, kLayoutSW128);
-              umma_f16_ss(dS, a, b, kIdS, acc);
-              acc = 1;
-            }
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t a = smem_desc(sbase + kOffQ + 4 * kQBlk + ks * 32, 16, 512, kLayoutSW64);
-            const uint64_t b = smem_desc(st + 4 * kKvBlk + ks * 32, 16, 512, kLayoutSW64);
-            umma_f16_ss(dS, a, b, kIdS, 1u);
-          }
-          umma_commit(bar(S_FULL + (g & 1)));
-          if (j == n_t - 1) umma_commit(bar(Q_EMPTY));
-        }
-        __syncwarp();
-        if (j > 0 && !(ok = issue_pv(g - 1, j == 1))) break;
+      for (int j = 0; ok && j < min(2, n_t); ++j) ok = issue_s(g0 + j, sg.t0 + j, L, j == n_t - 1);
+      for (int j = 0; ok && j < n_t; ++j) {
+        ok = issue_pv(g0 + j, j == 0);
+        if (ok && j + 2 < n_t) ok = issue_s(g0 + j + 2, sg.t0 + j + 2, L, j + 2 == n_t - 1);
       }
-      if (!ok) break;
-      if (!(ok = issue_pv(g - 1, n_t == 1))) break;
+      g0 += n_t;
       ++seg_i;
     }
     // every MMA issued by this thread has completed before TMEM is freed
@@ -300,8 +332,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t x_remote = mapa(x_local, peer);
     const uint32_t xfull_remote = mapa(bar(X_FULL), peer);
     const uint32_t xempty_remote = mapa(bar(X_EMPTY), peer);
-    const uint32_t p_row = sbase + kOffP + row * 128;
     const uint32_t sw = static_cast<uint32_t>(row & 7);
+    // PV_g has completed once the barrier of its P buffer finished the phase
+    // numbered g / 2 (each buffer sees every other tile)
+    auto wait_pv = [&](int g) -> bool {
+      return warp_wait(bar(PV_DONE + (g & 1)), (g >> 1) & 1, p.err);
+    };
     ChunkWalk walk;
     walk.init(p.tile_prefix, p.B, chunk, cs);
     Segment sg;
@@ -375,10 +411,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         l = l * alpha + sum;
 
-        // the previous P . C must be done before P is overwritten or O rescaled
-        if (j > 0 && !(ok = warp_wait(bar(PV_DONE), (g - 1) & 1, p.err))) break;
-        tc_fence_after();
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // P buffer g&1 was last read by PV_{g-2}; O may be rescaled only
+        // after PV_{g-1} (tiles of an earlier segment were all retired by
+        // that segment's epilogue)
+        if (j >= 2 && !(ok = wait_pv(g - 2))) break;
+        if (j >= 1 && __any_sync(0xffffffffu, resc)) {
+          if (!(ok = wait_pv(g - 1))) break;
+          tc_fence_after();
           for (int c0 = 0; c0 < kLatPerCta; c0 += 32) {
             float o[32];
             tmem_ld32(tmem + lane_base + kTmemO + c0, o);
@@ -387,21 +426,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
             tmem_st32(tmem + lane_base + kTmemO + c0, o);
           }
-          tmem_wait_st();
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          st_shared_v4(p_row + ((static_cast<uint32_t>(k) ^ sw) << 4), pk[4 * k], pk[4 * k + 1],
-                       pk[4 * k + 2], pk[4 * k + 3]);
-        fence_proxy_async_smem();
+        tc_fence_after();
+        tmem_st32u(tmem + lane_base + kTmemP + (g & 1) * 32, pk);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(P_FULL));
+        if (lane == 0) mbar_arrive(bar(P_FULL + (g & 1)));
       }
       if (!ok) break;
 
       // epilogue: u = O / l (this CTA's 256 columns), lse in natural log
-      if (!(ok = warp_wait(bar(PV_DONE), (g - 1) & 1, p.err))) break;
+      if (!(ok = wait_pv(g - 1))) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -510,9 +546,17 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   p.page_size = a.page_size;
   p.num_pages = a.num_pages;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  const dim3 grid(2 * a.num_chunks * a.s_q, 1, 1);
-  decode_sm100_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.num_chunks * a.s_q, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_sm100_kernel, p);
 }
 
 }  // namespace mla

@@ -83,8 +83,13 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
-// Per-head up-projection on the tensor cores (bf16).
-cudaError_t launch_up_proj_sm100(const void* u, const void* W_UV, void* o, int T, int n_h,
-                                 int d_c, int d_v, cudaStream_t s);
+// Per-head up-projection on the tensor cores (bf16, d_v = 128, d_c a
+// multiple of 64 up to 512).  w_map: W_UV as [n_h * 128, d_c], box 64 x 128,
+// 128-byte swizzle; u_map: u as [T, n_h, d_c], box 64 x 1 x
+// up_proj_sm100_box_rows(T), 128-byte swizzle.
+int up_proj_sm100_prepare();
+int up_proj_sm100_box_rows(int T);
+cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_map, void* o,
+                                 int* err, int T, int n_h, int d_c, cudaStream_t s);
 
 }  // namespace mla

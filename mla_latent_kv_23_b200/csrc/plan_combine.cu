@@ -10,6 +10,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -49,6 +50,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
                                                             int s_q, int max_len, int num_chunks,
                                                             int* header, int* tile_prefix,
                                                             int* split_base, int* err) {
+  // let the attend kernel start its prologue while this one runs
+  ptx::pdl_launch_dependents();
   __shared__ int warp_sums[32];
   int carry = 0, total = 0;
   for (int base = 0; base < B; base += blockDim.x) {
@@ -91,59 +94,81 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   }
 }
 
-constexpr int kCombineThreads = 128;
-constexpr int kCombineHeads = 4;  // heads per block
+constexpr int kCombineWarps = 8;
+constexpr int kCombineThreads = 32 * kCombineWarps;
 
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// One warp per output row (b, r, head).  Lane s holds the weight of split s
+// (32 at a time); the column loop broadcasts it with a shuffle, so every
+// split costs one exp per row and one float4 load per lane per 128 columns.
 template <bool kBf16>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const int* __restrict__ tile_prefix, const int* __restrict__ split_base,
                    const float* __restrict__ part_u, const float* __restrict__ part_lse,
                    void* __restrict__ u_out, float* __restrict__ lse_out, int s_q, int n_h,
-                   int d_c) {
-  const int b = blockIdx.x / s_q, r = blockIdx.x % s_q;
+                   int d_c, int rows) {
+  ptx::pdl_wait_previous();
+  ptx::pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int h = row % n_h, br = row / n_h;
+  const int b = br / s_q, r = br % s_q;
   const int nsplit = split_base[b + 1] - split_base[b];
   const bool empty = tile_prefix[b + 1] == tile_prefix[b];
   if (nsplit == 0 && !empty) return;  // written directly by the attend stage
-  const int h0 = blockIdx.y * kCombineHeads;
-  for (int h = h0; h < min(h0 + kCombineHeads, n_h); ++h) {
-    const size_t orow = (static_cast<size_t>(b) * s_q + r) * n_h + h;
-    float m = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) {
-      const size_t slot = static_cast<size_t>(split_base[b] + s) * s_q + r;
-      m = fmaxf(m, part_lse[slot * n_h + h]);
-    }
-    float z = 0.f;
-    if (m != -INFINITY)
-      for (int s = 0; s < nsplit; ++s) {
-        const size_t slot = static_cast<size_t>(split_base[b] + s) * s_q + r;
-        z += expf(part_lse[slot * n_h + h] - m);
-      }
-    const float lse_all = (m == -INFINITY) ? -INFINITY : m + logf(z);
-    for (int c = threadIdx.x * 4; c < d_c; c += kCombineThreads * 4) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (m != -INFINITY)
-        for (int s = 0; s < nsplit; ++s) {
-          const size_t slot = static_cast<size_t>(split_base[b] + s) * s_q + r;
-          const float w = expf(part_lse[slot * n_h + h] - lse_all);
+  const size_t slot0 = static_cast<size_t>(split_base[b]) * s_q + r;  // slot of split s: slot0 + s*s_q
+  float m = -INFINITY;
+  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, part_lse[(slot0 + (size_t)s * s_q) * n_h + h]);
+  m = warp_max(m);
+  float z = 0.f;
+  if (m != -INFINITY)
+    for (int s = lane; s < nsplit; s += 32) z += expf(part_lse[(slot0 + (size_t)s * s_q) * n_h + h] - m);
+  z = warp_sum(z);
+  const float lse_all = (m == -INFINITY) ? -INFINITY : m + logf(z);
+  for (int c = lane * 4; c < d_c; c += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (m != -INFINITY) {
+      for (int s0 = 0; s0 < nsplit; s0 += 32) {
+        const int s_me = s0 + lane;
+        const float w_me = s_me < nsplit
+            ? expf(part_lse[(slot0 + (size_t)s_me * s_q) * n_h + h] - lse_all) : 0.f;
+        const int n_here = min(32, nsplit - s0);
+#pragma unroll 4
+        for (int k = 0; k < n_here; ++k) {
+          const float w = __shfl_sync(0xffffffffu, w_me, k);
+          const size_t slot = slot0 + (size_t)(s0 + k) * s_q;
           const float4 v = *reinterpret_cast<const float4*>(part_u + (slot * n_h + h) * d_c + c);
           acc.x += w * v.x;
           acc.y += w * v.y;
           acc.z += w * v.z;
           acc.w += w * v.w;
         }
-      if (kBf16) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(u_out) + orow * d_c + c) = pk;
-      } else {
-        *reinterpret_cast<float4*>(static_cast<float*>(u_out) + orow * d_c + c) = acc;
       }
     }
-    if (lse_out != nullptr && threadIdx.x == 0) lse_out[orow] = lse_all;
+    const size_t orow = static_cast<size_t>(br) * n_h + h;
+    if (kBf16) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(u_out) + orow * d_c + c) = pk;
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(u_out) + orow * d_c + c) = acc;
+    }
   }
+  if (lse_out != nullptr && lane == 0) lse_out[static_cast<size_t>(br) * n_h + h] = lse_all;
 }
 
 }  // namespace
@@ -156,16 +181,23 @@ cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
-  dim3 grid(a.B * a.s_q, (a.n_h + kCombineHeads - 1) / kCombineHeads);
+  const int rows = a.B * a.s_q * a.n_h;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows + kCombineWarps - 1) / kCombineWarps, 1, 1);
+  cfg.blockDim = dim3(kCombineThreads, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (a.bf16)
-    combine_kernel<true><<<grid, kCombineThreads, 0, s>>>(a.tile_prefix, a.split_base, a.part_u,
-                                                          a.part_lse, a.u, a.lse, a.s_q, a.n_h,
-                                                          a.d_c);
-  else
-    combine_kernel<false><<<grid, kCombineThreads, 0, s>>>(a.tile_prefix, a.split_base, a.part_u,
-                                                           a.part_lse, a.u, a.lse, a.s_q, a.n_h,
-                                                           a.d_c);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, combine_kernel<true>, (const int*)a.tile_prefix,
+                              (const int*)a.split_base, (const float*)a.part_u,
+                              (const float*)a.part_lse, a.u, a.lse, a.s_q, a.n_h, a.d_c, rows);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<false>, (const int*)a.tile_prefix,
+                            (const int*)a.split_base, (const float*)a.part_u,
+                            (const float*)a.part_lse, a.u, a.lse, a.s_q, a.n_h, a.d_c, rows);
 }
 
 }  // namespace mla

@@ -57,7 +57,19 @@ def test_v3_shape_ragged(s_q, splits):
 
 @pytest.mark.parametrize("s_q,seqlens", [(1, (1, 64, 65, 128, 129)), (2, (2, 64, 65, 130, 3))])
 def test_length_edges(s_q, seqlens):
+    # one token, exactly one tile, one tile + 1, two tiles, two tiles + 1;
+    # judged on exact bf16 inputs (q from the generator) with the tight bound
     w = v3_small(s_q=s_q, B=len(seqlens), seqlens=seqlens, block_table="identity")
+    inp = synth.draw(w)
+    q = synth.random_q(w)
+    out = run_pipeline(w, inp, q=to_dev(q, w))
+    picks = [(b, r, i) for b in range(w.B) for r in range(s_q) for i in (0, 5, 64, 127)]
+    assert_tight(check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"]))
+
+
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_length_edges_through_query_formation(s_q):
+    w = v3_small(s_q=s_q, B=4, seqlens=(64, 65, 128, 129), block_table="identity")
     inp = synth.draw(w)
     out = run_pipeline(w, inp)
     assert_parity(check_expanded(w, inp, out, some_heads(w, heads_first=(0, 5, 127))))
