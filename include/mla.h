@@ -138,7 +138,7 @@ typedef struct {
   int page_size;            /* tokens per page, a positive multiple of 64                         */
   int max_pages_per_seq;    /* columns of block_table                                            */
   int num_pages;            /* pages in kv_cache                                                 */
-  float softmax_scale;      /* multiplies the scores before softmax, finite                       */
+  float softmax_scale;      /* multiplies the scores before softmax, finite and > 0               */
   mla_dtype dtype;          /* of q, kv_cache and u                                              */
   int num_splits;           /* KV chunks the whole batch is cut into; 0 = one per SM pair        */
 } mla_decode_params;

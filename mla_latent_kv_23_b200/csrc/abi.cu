@@ -102,7 +102,7 @@ mla_status validate_decode(const mla_decode_params* p) {
   if (p->max_pages_per_seq < 1 || p->num_pages < 1) return MLA_ERR_INVALID_ARG;
   if ((long long)p->num_pages * p->page_size > INT_MAX) return MLA_ERR_UNSUPPORTED;
   if ((long long)p->max_pages_per_seq * p->page_size > INT_MAX) return MLA_ERR_UNSUPPORTED;
-  if (!std::isfinite(p->softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale) || !(p->softmax_scale > 0.f)) return MLA_ERR_INVALID_ARG;
   if (!valid_dtype(p->dtype)) return MLA_ERR_INVALID_ARG;
   if (p->num_splits < 0) return MLA_ERR_INVALID_ARG;
   if (p->B == 0) return MLA_OK;

@@ -140,8 +140,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar(P_FULL + i), 4);
       mbar_init(bar(PV_DONE + i), 1);
     }
-    mbar_init(bar(X_FULL), 128);
-    mbar_init(bar(X_EMPTY), 128);
+    mbar_init(bar(X_FULL), 1);    // armed once per tile with the 32 KB the peer sends
+    mbar_init(bar(X_EMPTY), 4);   // one arrive per peer softmax warp
+    mbar_arrive_expect_tx(bar(X_FULL), kXBytes);   // tile 0
     mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(Q_EMPTY), 1);
     mbar_init(bar(MMA_FINAL), 1);
@@ -333,10 +334,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t xfull_remote = mapa(bar(X_FULL), peer);
     const uint32_t xempty_remote = mapa(bar(X_EMPTY), peer);
     const uint32_t sw = static_cast<uint32_t>(row & 7);
+    const float c_log2 = p.scale_log2;
     // PV_g has completed once the barrier of its P buffer finished the phase
     // numbered g / 2 (each buffer sees every other tile)
     auto wait_pv = [&](int g) -> bool {
       return warp_wait(bar(PV_DONE + (g & 1)), (g >> 1) & 1, p.err);
+    };
+    // Own partial S of tile g: TMEM -> registers, free the TMEM buffer, and
+    // send the row to the peer (st.async; the peer's barrier counts bytes).
+    auto fetch_and_send = [&](int g, float (&dst)[64]) -> bool {
+      if (!warp_wait(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err)) return false;
+      tc_fence_after();
+      {
+        float (&d0)[32] = *reinterpret_cast<float(*)[32]>(&dst[0]);
+        float (&d1)[32] = *reinterpret_cast<float(*)[32]>(&dst[32]);
+        const uint32_t ta = tmem + lane_base + kTmemS + (g & 1) * 64;
+        tmem_ld32(ta, d0);
+        tmem_ld32(ta + 32, d1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(S_EMPTY + (g & 1)));
+      // the peer has read what we sent for tile g - 1
+      if (!warp_wait<true>(bar(X_EMPTY), (g & 1) ^ 1, p.err)) return false;
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        st_async_v4(x_remote + ((static_cast<uint32_t>(k) ^ sw) << 4), dst[4 * k], dst[4 * k + 1],
+                    dst[4 * k + 2], dst[4 * k + 3], xfull_remote);
+      return true;
     };
     ChunkWalk walk;
     walk.init(p.tile_prefix, p.B, chunk, cs);
@@ -346,32 +372,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (ok && walk.next(sg)) {
       const int L = p.seqlens[sg.b];
       const int L_eff = L - p.s_q + 1 + qrow;  // positions this query row may see
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f, l_exact = 0.f;
       const int n_t = sg.t1 - sg.t0;
+      float s[64], s_next[64];
+      if (!(ok = fetch_and_send(g, s))) break;
       for (int j = 0; j < n_t; ++j, ++g) {
         const int t = sg.t0 + j;
-        float s[64];
-        if (!(ok = warp_wait(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
-        tc_fence_after();
-        {
-          float (&s0)[32] = *reinterpret_cast<float(*)[32]>(&s[0]);
-          float (&s1)[32] = *reinterpret_cast<float(*)[32]>(&s[32]);
-          const uint32_t ta = tmem + lane_base + kTmemS + (g & 1) * 64;
-          tmem_ld32(ta, s0);
-          tmem_ld32(ta + 32, s1);
-          tmem_wait_ld();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(S_EMPTY + (g & 1)));
-
-        // exchange partial scores with the peer CTA
-        if (!(ok = warp_wait<true>(bar(X_EMPTY), (g & 1) ^ 1, p.err))) break;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          st_cluster_v4(x_remote + ((static_cast<uint32_t>(k) ^ sw) << 4), s[4 * k], s[4 * k + 1],
-                        s[4 * k + 2], s[4 * k + 3]);
-        mbar_arrive_remote(xfull_remote);
+        // (1) the peer's partial of this tile; S = own + peer (fp32 addition
+        // commutes, so both CTAs hold the same S)
         if (!(ok = warp_wait<true>(bar(X_FULL), g & 1, p.err))) break;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -381,35 +389,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           s[4 * k + 2] += v.z;
           s[4 * k + 3] += v.w;
         }
-        mbar_arrive_remote(xempty_remote);
+        if (threadIdx.x == kWarpSoftmax0 * 32) mbar_arrive_expect_tx(bar(X_FULL), kXBytes);  // tile g + 1
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(xempty_remote);
+        // (2) start the next tile's exchange before this tile's arithmetic
+        if (j + 1 < n_t && !(ok = fetch_and_send(g + 1, s_next))) break;
 
-        // masked online softmax in log2 units
+        // (3) masked online softmax in log2 units
         const int nv = L_eff - t * kTileTokens;
-        float mx = -INFINITY;
+        if (nv < kTileTokens) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x = c < nv ? s[c] * p.scale_log2 : -INFINITY;
-          s[c] = x;
-          mx = fmaxf(mx, x);
+          for (int c = 0; c < 64; ++c)
+            if (c >= nv) s[c] = -INFINITY;
         }
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_log2;  // scale > 0
         const float m_new = fmaxf(m, mx);
         const bool resc = m_new > m + kRescaleThreshold;
         float alpha = 1.f;
         if (resc) {
-          alpha = exp2f(m - m_new);
+          alpha = ex2_approx(m - m_new);
           m = m_new;
         }
-        const float m_use = m == -INFINITY ? 0.f : m;
-        float sum = 0.f;
+        const float neg_m = m == -INFINITY ? 0.f : -m;
+        float r0 = 0.f, r1 = 0.f, e0 = 0.f, e1 = 0.f;
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(exp2f(s[c] - m_use), exp2f(s[c + 1] - m_use));
+          const float a = ex2_approx(fmaf(s[c], c_log2, neg_m));
+          const float b = ex2_approx(fmaf(s[c + 1], c_log2, neg_m));
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
           const float2 pf = __bfloat1622float2(pr);
-          sum += pf.x + pf.y;
+          if (c & 2) { r1 += pf.x + pf.y; e1 += a + b; } else { r0 += pf.x + pf.y; e0 += a + b; }
           pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        l = l * alpha + sum;
+        // u is normalised by the sum of the rounded weights it was built
+        // from; lse uses the unrounded weights
+        l = l * alpha + (r0 + r1);
+        l_exact = l_exact * alpha + (e0 + e1);
 
         // P buffer g&1 was last read by PV_{g-2}; O may be rescaled only
         // after PV_{g-1} (tiles of an earlier segment were all retired by
@@ -433,6 +457,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(P_FULL + (g & 1)));
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = s_next[c];
       }
       if (!ok) break;
 
@@ -440,7 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!(ok = wait_pv(g - 1))) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const float lse = l_exact > 0.f ? (m + log2f(l_exact)) * 0.69314718055994531f : -INFINITY;
       const bool write = row < p.n_h;
       const size_t orow = (size_t)(sg.b * p.s_q + qrow) * p.n_h + row;
       const size_t slot = sg.whole ? 0 : (size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow;

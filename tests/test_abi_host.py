@@ -54,6 +54,7 @@ def params(**kw):
     (dict(d_R=7), INVALID), (dict(d_R=128), UNSUPPORTED), (dict(page_size=63), INVALID),
     (dict(page_size=0), INVALID), (dict(max_pages_per_seq=0), INVALID), (dict(num_pages=0), INVALID),
     (dict(softmax_scale=float("nan")), INVALID), (dict(softmax_scale=float("inf")), INVALID),
+    (dict(softmax_scale=0.0), INVALID), (dict(softmax_scale=-0.1), INVALID),
     (dict(dtype=7), INVALID), (dict(num_splits=-1), INVALID), (dict(B=-1), INVALID),
     (dict(q=None), INVALID), (dict(kv_cache=None), INVALID), (dict(u=None), INVALID),
     (dict(block_table=None), INVALID), (dict(seqlens=None), INVALID),
