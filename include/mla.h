@@ -168,6 +168,27 @@ mla_status mla_decode_attend(const mla_decode_params* p, void* workspace, size_t
 mla_status mla_decode_combine(const mla_decode_params* p, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/*
+ * mla_decode without a caller-provided workspace.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory, such as a host framework that owns all device memory and
+ * hands a kernel library only inputs and outputs (a fixed serving pool, a
+ * plugin interface without a workspace argument).
+ *
+ * Same parameters, results and errors as mla_decode.  The scratch space is
+ * a 32 MiB array inside the library (a file-scope __device__ variable): every
+ * GPU that loads the library holds it until the process exits, and this call
+ * allocates nothing.  Parameters whose mla_decode_workspace_size exceeds
+ * 32 MiB are rejected with MLA_ERR_WORKSPACE_TOO_SMALL before anything is
+ * enqueued.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls on a device share the array and
+ * leave their data in it; nothing in it needs to start at zero, but calls
+ * whose work overlaps on the GPU race on it, so order them on one stream or
+ * with events.
+ */
+mla_status mla_decode_noalloc(const mla_decode_params* p, void* stream);
+
 /* Which attend kernel these parameters select: 1 = tensor-core (tcgen05)
  * kernel, 0 = CUDA-core kernel; and the number of KV chunks it will use. */
 mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_cores,

@@ -53,6 +53,7 @@ SIGNATURES = {
     "mla_decode_attend": ([_P, _V, _S, _V], _I),
     "mla_decode_combine": ([_P, _V, _S, _V], _I),
     "mla_decode_kernel_info": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    "mla_decode_noalloc": ([_P, _V], _I),
     "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _V], _I),
     "mla_check_device_errors": ([_V, ctypes.POINTER(_I)], _I),
 }
@@ -196,6 +197,12 @@ def mla_decode_attend(p: DecodeParams, workspace, stream=None) -> None:
 
 def mla_decode_combine(p: DecodeParams, workspace, stream=None) -> None:
     _stage("mla_decode_combine", p, workspace, stream)
+
+
+def mla_decode_noalloc(p: DecodeParams, stream=None) -> None:
+    """mla_decode with the library's own fixed scratch array (no workspace
+    argument, no allocation); see include/mla.h for its size limit."""
+    _check(lib().mla_decode_noalloc(ctypes.byref(p), _stream(stream)), "mla_decode_noalloc")
 
 
 def mla_up_proj(u, W_UV, o, stream=None) -> None:
