@@ -184,12 +184,9 @@ mla_status encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t r
 mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s) {
   if (!r.tc) return cuda_status(launch_decode_simt(r.a, s));
   Sm100Maps maps;
-  const uint64_t qrows = (uint64_t)p->B * p->s_q * p->n_h;
   const uint64_t kvrows = (uint64_t)p->num_pages * p->page_size;
   mla_status st;
-  if ((st = encode_2d(&maps.q_lat, p->q, 576, qrows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
-      (st = encode_2d(&maps.q_rope, p->q, 576, qrows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK ||
-      (st = encode_2d(&maps.kv_lat, p->kv_cache, 576, kvrows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+  if ((st = encode_2d(&maps.kv_lat, p->kv_cache, 576, kvrows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
       (st = encode_2d(&maps.kv_rope, p->kv_cache, 576, kvrows, 32, 64, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
     return st;
   return cuda_status(launch_decode_sm100(r.a, maps, s));

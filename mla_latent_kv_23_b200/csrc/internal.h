@@ -46,10 +46,10 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s);
 
 // Tensor-core decode for n_h <= 128, d_c = 512, d_R = 64, bf16.
-// maps: q latent (box 64x128, SW128), q rope (32x128, SW64),
-//       kv latent (64x64, SW128), kv rope (32x64, SW64).
+// maps over the cache [rows, 576]: latent boxes 64 x 64 (128-byte swizzle),
+// RoPE boxes 32 x 64 (64-byte swizzle).
 struct Sm100Maps {
-  CUtensorMap q_lat, q_rope, kv_lat, kv_rope;
+  CUtensorMap kv_lat, kv_rope;
 };
 cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s);
 size_t decode_sm100_smem_bytes();
