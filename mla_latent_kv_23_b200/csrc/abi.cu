@@ -181,6 +181,19 @@ mla_status encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t r
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// 3D map over the queries [B * s_q, n_h, 576] (bf16), box box_x x 16 heads x 1.
+mla_status encode_q(CUtensorMap* m, const void* ptr, uint64_t n_h, uint64_t qrows, uint32_t box_x,
+                    CUtensorMapSwizzle sw) {
+  const cuuint64_t dims[3] = {576, n_h, qrows};
+  const cuuint64_t strides[2] = {576 * 2, n_h * 576 * 2};
+  const cuuint32_t box[3] = {box_x, 16, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s) {
   if (!r.tc) return cuda_status(launch_decode_simt(r.a, s));
   Sm100Maps maps;
@@ -188,6 +201,10 @@ mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s)
   mla_status st;
   if ((st = encode_2d(&maps.kv_lat, p->kv_cache, 576, kvrows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
       (st = encode_2d(&maps.kv_rope, p->kv_cache, 576, kvrows, 32, 64, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+    return st;
+  const uint64_t qrows = (uint64_t)p->B * p->s_q;
+  if ((st = encode_q(&maps.q_lat, p->q, p->n_h, qrows, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+      (st = encode_q(&maps.q_rope, p->q, p->n_h, qrows, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
     return st;
   return cuda_status(launch_decode_sm100(r.a, maps, s));
 }

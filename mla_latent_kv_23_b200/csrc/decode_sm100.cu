@@ -3,42 +3,56 @@
 //
 // Math ("MLA deep compression", absorption section, both equations, and its
 // decoupled-RoPE section): all heads of one query row share every cached row
-// [c || k^R], so the 128 heads are the M dimension of two dense contractions
-// per 64-token tile:
-//     S = Q . [C || K^R]^T      (M = 128, N = 64 tokens, K = 576)
-//     O = O * alpha + P . C     (M = 128, N = 512 latent, K = 64 tokens)
+// [c || k^R], so the heads are the M dimension of two dense contractions per
+// 64-token tile,
+//     S = Q . [C || K^R]^T      (K = 576)
+//     O = O * alpha + P . C     (N = 512 latent)
 // with an online softmax between them; u = O / l at the end.
 //
-// Column split.  O for 128 heads x 512 latent in fp32 fills all 512 TMEM
-// columns, which leaves no room for S.  So a cluster of two CTAs splits the
-// columns: CTA r owns latent columns [256r, 256r + 256) and RoPE columns
-// [32r, 32r + 32).  Each CTA loads only its own columns of every cache tile
-// (each byte is read from HBM once) and computes a partial S over its 288
-// columns; the partial S tiles are swapped with one 32 KB bulk copy each way
-// per tile (completing on the receiver's transaction-count barrier), and both
-// CTAs add own + peer.  fp32 addition commutes, so both hold the same S, make
-// bit-identical softmax decisions, and each accumulates its own half of
-// O = P . C (N = 256).
+// A pair of CTAs (one 2-CTA cluster) shares every tile, and all tensor-core
+// work is paired (tcgen05 cta_group::2, issued by the even CTA):
+//  * Loads are split by columns.  CTA r loads, for every cached row, latent
+//    columns [128r, 128r + 128) and [256 + 128r, 256 + 128r + 128) plus RoPE
+//    columns [32r, 32r + 32): 288 of the 576 values, so each cache byte is
+//    read from HBM by exactly one SM and never re-read.
+//  * Output rows are split by heads: CTA r owns heads [64r, 64r + 64) and
+//    holds their O (64 heads x 512 latent, fp32) in its TMEM.
+//  * P . C is one paired MMA per 16 tokens and 256 latent columns
+//    (M = 128: 64 P rows from each CTA; N = 256: each CTA supplies the 128 of
+//    those columns it loaded).  The pair's tensor cores move the B halves
+//    between the SMs, so no latent data crosses shared memory.
+//  * S needs all 576 columns of a row, but each CTA holds only half of them.
+//    A paired MMA with M = 256, N = 128 computes, in CTA r, rows
+//    (head h, half j) = Q[h, columns of CTA j] against B = [CTA 0's columns of
+//    the 64 tokens | CTA 1's columns of the same tokens].  Row (h, j) is
+//    meaningful against CTA j's half of N, so TMEM lane (h, 0) holds the
+//    partial score over CTA 0's columns and lane (h, 1) the partial over
+//    CTA 1's columns; the other half of each row is discarded.  Lanes are
+//    ordered (32q + 16j + i) <-> head 16q + i, so the two partials of a head
+//    sit 16 lanes apart in one warp and one shuffle adds them.  Half of the
+//    S arithmetic is thrown away; in exchange nothing but barrier arrivals
+//    passes between the CTAs.
 //
-// TMEM per CTA (512 columns): O 256 | S 2 x 64 | Q latent 128 (bf16 pairs).
-// Shared memory: 3 tile stages of 36 KB, the query's RoPE columns (8 KB), two
-// P buffers (16 KB each), one receive and one send buffer for partial S
-// (32 KB each).  One shared-memory copy of a tile serves both contractions: a
-// TMA load with 128-byte swizzle writes each 64-column block as 64 rows x
-// 128 B, the K-major operand layout of S = Q K^T and the MN-major operand
-// layout of O = P C at the same time.
+// TMEM per CTA (512 columns): S 2 x 128 (double-buffered) | O 256.
+// Shared memory per CTA: Q (128 rows x 288 values, the S operand A) 72 KB;
+// 3 tile stages of 36 KB; two P buffers (64 heads x 64 tokens bf16) of 8 KB.
+// One shared-memory copy of a tile serves both contractions: a TMA load with
+// 128-byte swizzle writes each 64-column block as 64 rows x 128 B, the
+// K-major layout of the S operand and the MN-major layout of the P . C
+// operand at the same time.
 //
-// Roles (384 threads): warp 0 = TMA producer (the whole warp prefetches
-// block-table entries, lane 0 issues copies); warp 1 = MMA issuer, which
-// issues S or P . C for whichever tile is ready (S runs up to two tiles
-// ahead) and zeroes cache rows past a sequence's end; warp 2 = TMEM
-// allocator; warp 3 = exchange: ships each partial S to the peer, tells the
-// peer when its last shipment has been read, arms the receive barrier;
-// warps 4-11 = softmax: warp 4 + 4h + q serves TMEM lanes [32q, 32q + 32)
-// (head rows) and tile columns [32h, 32h + 32), so each head row has two
-// threads sharing the row maximum through shared memory.  Per tile the
-// softmax warps (1) add the peer's partial of tile g, (2) stage their
-// partial of tile g + 1 for the exchange warp, (3) do tile g's arithmetic.
+// Roles (384 threads): warp 0 = TMA producer for this CTA's columns (the
+// whole warp prefetches block-table entries, lane 0 issues copies); warp 1 =
+// MMA issuer (even CTA only): S for whichever tile is ready (up to two tiles
+// ahead), P . C as soon as P is ready; warp 2 = TMEM allocator; warp 3 =
+// relay: loads the segment's query by TMA, zeroes cache rows past a
+// sequence's end in this CTA's stage, and signals the even CTA's barriers
+// that this CTA's operands are in place; warps 4-11 = softmax: warp 4 + 4c + q
+// reads TMEM lanes [32q, 32q + 32) and tokens [32c, 32c + 32) of a tile.
+// Each thread finishes 16 scores of one head; the row maximum is shared
+// through shared memory with one 8-warp rendezvous per tile.  O rows are
+// rescaled by the warp that can reach their TMEM lanes, which derives the
+// same maximum from the same shared values.
 //
 // Work: the plan stage cuts the batch's tiles into equal chunks; cluster c
 // handles chunk c / s_q for query row c % s_q, walking its segments in order.
@@ -54,43 +68,38 @@ namespace {
 using namespace ptx;
 
 constexpr int kThreads = 384;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpAlloc = 2, kWarpXchg = 3, kWarpSoftmax0 = 4;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpAlloc = 2, kWarpRelay = 3, kWarpSoftmax0 = 4;
 constexpr int kStages = 3;
-constexpr int kDc = 512, kWidth = 576;
-constexpr int kLatPerCta = 256, kRopePerCta = 32;
+constexpr int kDc = 512;
 
 constexpr uint32_t kKvBlk = 64 * 128;                    // tile: 64 rows x 64 cols, SW128
 constexpr uint32_t kKvRope = 64 * 64;                    // tile: 64 rows x 32 cols, SW64
 constexpr uint32_t kStageBytes = 4 * kKvBlk + kKvRope;   // 36864
-constexpr uint32_t kQRopeBytes = 128 * 64;               // 128 rows x 32 cols bf16, SW64
-constexpr uint32_t kPBytes = 128 * 128;                  // 128 rows x 64 tokens bf16, SW128
-constexpr uint32_t kXBytes = 128 * 256;                  // one partial S: 128 x 64 fp32
+constexpr uint32_t kQBlk = 128 * 128;                    // Q: 128 rows x 64 cols, SW128
+constexpr uint32_t kQRope = 128 * 64;                    // Q: 128 rows x 32 cols, SW64
+constexpr uint32_t kQBytes = 4 * kQBlk + kQRope;         // 73728
+constexpr uint32_t kPBytes = 64 * 128;                   // 64 heads x 64 tokens bf16, SW128
 
-constexpr uint32_t kOffKv = 0;
-constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;    // [2]
-constexpr uint32_t kOffQRope = kOffP + 2 * kPBytes;
-constexpr uint32_t kOffXin = kOffQRope + kQRopeBytes;
-constexpr uint32_t kOffXout = kOffXin + kXBytes;
-constexpr uint32_t kOffRed = kOffXout + kXBytes;              // float [2][2][128] row maxima
-constexpr uint32_t kOffSum = kOffRed + 2 * 2 * 128 * 4;       // float [2][2][128] row sums
-constexpr uint32_t kOffBar = kOffSum + 2 * 2 * 128 * 4;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKv = kOffQ + kQBytes;
+constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;   // [2]
+constexpr uint32_t kOffRed = kOffP + 2 * kPBytes;            // float [2 parity][2 c][64 heads]
+constexpr uint32_t kOffSum = kOffRed + 2 * 2 * 64 * 4;       // float [2 kind][2 c][64 heads]
+constexpr uint32_t kOffBar = kOffSum + 2 * 2 * 64 * 4;
 
 enum Bar {
-  KV_FULL = 0,
-  KV_EMPTY = KV_FULL + kStages,
-  S_FULL = KV_EMPTY + kStages,   // [2] per S buffer
-  S_EMPTY = S_FULL + 2,          // [2]
-  P_FULL = S_EMPTY + 2,          // [2] per P buffer
-  PV_DONE = P_FULL + 2,          // [2]
-  X_FULL = PV_DONE + 2,          // peer's partial S landed in our receive buffer
-  X_EMPTY,                       // peer has read what we sent last
-  X_READ,                        // our softmax warps have read the receive buffer
-  X_OUT_READY,                   // our softmax warps have staged the send buffer
-  X_OUT_FREE,                    // the last send has left the send buffer
-  Q_FULL,
-  Q_EMPTY,
-  SM_PAIR,                       // [4] the two softmax warps sharing a TMEM lane quarter
-  MMA_FINAL = SM_PAIR + 4,
+  LOCAL_FULL = 0,                  // [3] this CTA's TMA bytes of a stage
+  KV_FULL = LOCAL_FULL + kStages,  // [3] even CTA: both CTAs' stage ready (2 relay arrivals)
+  KV_EMPTY = KV_FULL + kStages,    // [3] P . C of the stage's tile done (paired commit)
+  S_FULL = KV_EMPTY + kStages,     // [2] per S buffer (paired commit)
+  S_EMPTY = S_FULL + 2,            // [2] even CTA: 16 softmax warps read the S buffer
+  P_FULL = S_EMPTY + 2,            // [2] even CTA: 16 softmax warps wrote P
+  PV_DONE = P_FULL + 2,            // [2] (paired commit)
+  Q_LOCAL = PV_DONE + 2,           // this CTA's query bytes
+  Q_FULL,                          // even CTA: both queries in place (2 relay arrivals)
+  Q_EMPTY,                         // last S of a segment done (paired commit)
+  GRP,                             // the 8 softmax warps of this CTA
+  MMA_FINAL,
   BAR_COUNT
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + BAR_COUNT * 8;
@@ -98,17 +107,22 @@ constexpr uint32_t kSmemUsed = kOffTmemSlot + 16;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 0;     // 256 columns
-constexpr uint32_t kTmemS = 256;   // 2 x 64 columns
-constexpr uint32_t kTmemQ = 384;   // 128 columns: the 256 latent query values per row
+constexpr uint32_t kTmemS = 0;     // 2 x 128 columns
+constexpr uint32_t kTmemO = 256;   // 2 x 128 columns (latent blocks 0-255, 256-511)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
+constexpr uint16_t kBothCtas = 3;
 
-static_assert(kStageBytes % 1024 == 0 && kOffP % 1024 == 0 && kOffQRope % 1024 == 0, "align");
+static_assert(kOffKv % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "align");
 static_assert(kSmemBytes <= 232448, "shared memory");
+
+// First latent column of 64-column block kc (0..3) of the columns CTA `half`
+// owns; the RoPE columns of that CTA start at 512 + 32 half.
+__device__ __forceinline__ int lat_col(int kc, int half) {
+  return (kc >> 1) * 256 + half * 128 + (kc & 1) * 64;
+}
 
 struct Params {
   Sm100Maps maps;
-  const __nv_bfloat16* q;
   const int* block_table;
   const int* seqlens;
   const int* header;
@@ -136,46 +150,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (sbase - raw_addr);
-  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cid = blockIdx.x >> 1;
   const int chunk = cid / p.s_q, qrow = cid % p.s_q;
   auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * i; };
+  // barriers that live in the even CTA, addressed from either CTA
+  auto lead_bar = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(KV_FULL + s), 1);
+      mbar_init(bar(LOCAL_FULL + s), 1);
+      mbar_init(bar(KV_FULL + s), 2);
       mbar_init(bar(KV_EMPTY + s), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(S_FULL + i), 1);
-      mbar_init(bar(S_EMPTY + i), 8);   // one arrive per softmax warp
-      mbar_init(bar(P_FULL + i), 8);
+      mbar_init(bar(S_EMPTY + i), 16);
+      mbar_init(bar(P_FULL + i), 16);
       mbar_init(bar(PV_DONE + i), 1);
     }
-    mbar_init(bar(X_FULL), 1);                      // armed with the 32 KB of one tile
-    mbar_arrive_expect_tx(bar(X_FULL), kXBytes);    // tile 0
-    mbar_init(bar(X_EMPTY), 1);
-    mbar_init(bar(X_READ), 8);
-    mbar_init(bar(X_OUT_READY), 8);
-    mbar_init(bar(X_OUT_FREE), 1);
-    mbar_init(bar(Q_FULL), 8);
+    mbar_init(bar(Q_LOCAL), 1);
+    mbar_init(bar(Q_FULL), 2);
     mbar_init(bar(Q_EMPTY), 1);
-    for (int i = 0; i < 4; ++i) mbar_init(bar(SM_PAIR + i), 2);
+    mbar_init(bar(GRP), 8);
     mbar_init(bar(MMA_FINAL), 1);
     fence_mbar_init();
   }
   if (warp == kWarpAlloc) {
-    tmem_alloc(sbase + kOffTmemSlot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(sbase + kOffTmemSlot, kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == kWarpTma && lane == 0) {
     prefetch_tmap(&p.maps.kv_lat);
     prefetch_tmap(&p.maps.kv_rope);
   }
+  if (warp == kWarpRelay && lane == 0) {
+    prefetch_tmap(&p.maps.q_lat);
+    prefetch_tmap(&p.maps.q_rope);
+  }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // the peer's barriers exist before anything is sent to them
+  cluster_sync();  // both CTAs' barriers and TMEM exist before either uses the other's
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base + kOffTmemSlot);
   // everything above overlaps the plan kernel; its results are read below
@@ -209,17 +226,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int page = __shfl_sync(0xffffffffu, my_page, i);
           if (lane == 0) {
             const int s = g % kStages, n = g / kStages;
-            ok = mbar_wait(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT);
+            ok = mbar_wait<true>(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT);
             if (ok) {
               const int tok = (t0 + i) * kTileTokens;
               const int y = page * p.page_size + tok % p.page_size;
               const uint32_t st = sbase + kOffKv + s * kStageBytes;
-              mbar_arrive_expect_tx(bar(KV_FULL + s), kStageBytes);
-              for (int kb = 0; kb < 4; ++kb)
-                tma_load_2d(st + kb * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
-                            rank * kLatPerCta + kb * 64, y);
-              tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(KV_FULL + s),
-                          kDc + rank * kRopePerCta, y);
+              mbar_arrive_expect_tx(bar(LOCAL_FULL + s), kStageBytes);
+              for (int kc = 0; kc < 4; ++kc)
+                tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(LOCAL_FULL + s),
+                            lat_col(kc, (int)rank), y);
+              tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(LOCAL_FULL + s),
+                          kDc + 32 * (int)rank, y);
               last_n[s] = n;
             }
           }
@@ -231,410 +248,420 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // wait for this thread's own copies in flight before the CTA may exit
     if (lane == 0)
       for (int s = 0; s < kStages; ++s)
-        if (last_n[s] >= 0) mbar_wait(bar(KV_FULL + s), last_n[s] & 1, p.err, MLA_DEVFLAG_TIMEOUT);
+        if (last_n[s] >= 0) mbar_wait(bar(LOCAL_FULL + s), last_n[s] & 1, p.err, MLA_DEVFLAG_TIMEOUT);
+    __syncwarp();
+  } else if (warp == kWarpRelay) {
+    // ------------------------------------------------------------ relay
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.B, chunk, cs);
+    Segment sg;
+    int g = 0, seg_i = 0;
+    bool ok = true;
+    bool q_in_flight = false;
+    while (ok && walk.next(sg)) {
+      // this segment's query rows (h, j) = Q[64 rank + 16 qd + i, columns of
+      // CTA j], stored as row 32 qd + 16 j + i; heads >= n_h read as zero
+      // (the tensor map ends there)
+      if (seg_i > 0 && !(ok = warp_wait<true>(bar(Q_EMPTY), (seg_i - 1) & 1, p.err))) break;
+      if (lane == 0) {
+        const int z = sg.b * p.s_q + qrow;
+        mbar_arrive_expect_tx(bar(Q_LOCAL), kQBytes);
+        for (int qd = 0; qd < 4; ++qd)
+          for (int j = 0; j < 2; ++j) {
+            const int y = 64 * (int)rank + 16 * qd;
+            const uint32_t r0 = static_cast<uint32_t>(32 * qd + 16 * j);
+            for (int kc = 0; kc < 4; ++kc)
+              tma_load_3d(sbase + kOffQ + kc * kQBlk + r0 * 128, &p.maps.q_lat, bar(Q_LOCAL),
+                          lat_col(kc, j), y, z);
+            tma_load_3d(sbase + kOffQ + 4 * kQBlk + r0 * 64, &p.maps.q_rope, bar(Q_LOCAL),
+                        kDc + 32 * j, y, z);
+          }
+      }
+      q_in_flight = true;
+      if (!(ok = warp_wait(bar(Q_LOCAL), seg_i & 1, p.err))) break;
+      q_in_flight = false;
+      if (lane == 0) mbar_arrive_remote(lead_bar(Q_FULL));
+      __syncwarp();
+
+      const int L = p.seqlens[sg.b];
+      for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+        const int s = g % kStages;
+        if (!(ok = warp_wait(bar(LOCAL_FULL + s), (g / kStages) & 1, p.err))) break;
+        const int rows_valid = L - t * kTileTokens;
+        if (rows_valid < kTileTokens) {
+          // rows past the sequence end may hold anything; make them zero so
+          // that 0-probability x garbage cannot turn into NaN in P . C
+          uint8_t* tile = base + kOffKv + s * kStageBytes;
+          for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
+            if (lane < 8)
+              for (int kb = 0; kb < 4; ++kb)
+                *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
+                    make_uint4(0, 0, 0, 0);
+            if (lane < 4)
+              *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(lead_bar(KV_FULL + s));
+        __syncwarp();
+      }
+      ++seg_i;
+    }
+    // a query copy still in flight must land before the CTA may exit
+    if (q_in_flight && lane == 0) mbar_wait(bar(Q_LOCAL), seg_i & 1, p.err, MLA_DEVFLAG_TIMEOUT);
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t kIdS = idesc_bf16(128, 64, false);
-    constexpr uint32_t kIdPV = idesc_bf16(128, kLatPerCta, true);
-    ChunkWalk walk;
-    walk.init(p.tile_prefix, p.B, chunk, cs);
-    Segment sg;
-    int g0 = 0, seg_i = 0;
-    bool ok = true;
-    // S = Q . tile^T for global tile g (tile index t of the segment's sequence)
-    auto issue_s = [&](int g, int t, int L, bool last) {
-      const int s = g % kStages;
-      const int rows_valid = L - t * kTileTokens;
-      if (rows_valid < kTileTokens) {
-        // rows past the sequence end may hold anything; make them zero so
-        // that 0-probability x garbage cannot turn into NaN in P . C
-        uint8_t* tile = base + kOffKv + s * kStageBytes;
-        for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
-          if (lane < 8)
-            for (int kb = 0; kb < 4; ++kb)
-              *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
-                  make_uint4(0, 0, 0, 0);
-          if (lane < 4)
-            *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
-                make_uint4(0, 0, 0, 0);
+    if (leader) {
+      constexpr uint32_t kIdS = idesc_bf16(256, 128, false);
+      constexpr uint32_t kIdPV = idesc_bf16(128, 256, true);
+      ChunkWalk walk;
+      walk.init(p.tile_prefix, p.B, chunk, cs);
+      Segment sg;
+      int g0 = 0, seg_i = 0;
+      bool ok = true;
+      // S for global tile g: 16 steps over the latent columns, 2 over RoPE
+      auto issue_s = [&](int g, bool last) {
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t st = sbase + kOffKv + (g % kStages) * kStageBytes;
+          const uint32_t dS = tmem + kTmemS + (g & 1) * 128;
+          uint32_t acc = 0;
+          for (int kc = 0; kc < 4; ++kc)
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t a =
+                  smem_desc(sbase + kOffQ + kc * kQBlk + ks * 32, 16, 1024, kLayoutSW128);
+              const uint64_t b = smem_desc(st + kc * kKvBlk + ks * 32, 16, 1024, kLayoutSW128);
+              umma_f16_ss_pair(dS, a, b, kIdS, acc);
+              acc = 1;
+            }
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t a = smem_desc(sbase + kOffQ + 4 * kQBlk + ks * 32, 16, 512, kLayoutSW64);
+            const uint64_t b = smem_desc(st + 4 * kKvBlk + ks * 32, 16, 512, kLayoutSW64);
+            umma_f16_ss_pair(dS, a, b, kIdS, 1u);
+          }
+          umma_commit_pair(bar(S_FULL + (g & 1)), kBothCtas);
+          if (last) umma_commit_pair(bar(Q_EMPTY), kBothCtas);
         }
-        fence_proxy_async_smem();
         __syncwarp();
-      }
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t st = sbase + kOffKv + s * kStageBytes;
-        const uint32_t dS = tmem + kTmemS + (g & 1) * 64;
-        uint32_t acc = 0;
-        for (int kb = 0; kb < 4; ++kb)
-          for (int ks = 0; ks < 4; ++ks) {  // 16 columns per MMA, A from TMEM
-            const uint64_t b = smem_desc(st + kb * kKvBlk + ks * 32, 16, 1024, kLayoutSW128);
-            umma_f16_ts(dS, tmem + kTmemQ + (kb * 4 + ks) * 8, b, kIdS, acc);
-            acc = 1;
+      };
+      // O (+)= P . C for global tile g; `first` = first tile of its segment
+      auto issue_pv = [&](int g, bool first) {
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t st = sbase + kOffKv + (g % kStages) * kStageBytes;
+          const uint32_t pa = sbase + kOffP + (g & 1) * kPBytes;
+          for (int blk = 0; blk < 2; ++blk)
+            for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
+              const uint64_t a = smem_desc(pa + kk * 32, 16, 1024, kLayoutSW128);
+              const uint64_t b =
+                  smem_desc(st + 2 * blk * kKvBlk + kk * 2048, kKvBlk, 1024, kLayoutSW128);
+              umma_f16_ss_pair(tmem + kTmemO + blk * 128, a, b, kIdPV,
+                               (first && kk == 0) ? 0u : 1u);
+            }
+          umma_commit_pair(bar(KV_EMPTY + g % kStages), kBothCtas);
+          umma_commit_pair(bar(PV_DONE + (g & 1)), kBothCtas);
+        }
+        __syncwarp();
+      };
+      while (ok && walk.next(sg)) {
+        if (!(ok = warp_wait<true>(bar(Q_FULL), seg_i & 1, p.err))) break;
+        const int n_t = sg.t1 - sg.t0;
+        int s_next = 0, pv_next = 0;
+        uint64_t t_idle = 0;
+        while (pv_next < n_t) {
+          // P . C first when its P is ready (it frees a stage and a P buffer);
+          // otherwise S for the next tile whose data and S buffer are ready
+          bool did = false;
+          if (pv_next < s_next) {
+            const int g = g0 + pv_next;
+            bool ready = false;
+            if (lane == 0) ready = mbar_test_nb_cluster(bar(P_FULL + (g & 1)), (g >> 1) & 1);
+            if (__shfl_sync(0xffffffffu, ready, 0)) {
+              if (!(ok = warp_wait<true>(bar(P_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
+              issue_pv(g, pv_next == 0);
+              ++pv_next;
+              did = true;
+            }
           }
-        for (int ks = 0; ks < 2; ++ks) {  // RoPE columns, A from shared memory
-          const uint64_t a = smem_desc(sbase + kOffQRope + ks * 32, 16, 512, kLayoutSW64);
-          const uint64_t b = smem_desc(st + 4 * kKvBlk + ks * 32, 16, 512, kLayoutSW64);
-          umma_f16_ss(dS, a, b, kIdS, 1u);
-        }
-        umma_commit(bar(S_FULL + (g & 1)));
-        if (last) umma_commit(bar(Q_EMPTY));
-      }
-      __syncwarp();
-    };
-    // O (+)= P . C for global tile g; `first` = first tile of its segment
-    auto issue_pv = [&](int g, bool first) {
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t st = sbase + kOffKv + (g % kStages) * kStageBytes;
-        const uint32_t pa = sbase + kOffP + (g & 1) * kPBytes;
-        for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
-          const uint64_t a = smem_desc(pa + kk * 32, 16, 1024, kLayoutSW128);
-          const uint64_t b = smem_desc(st + kk * 2048, kKvBlk, 1024, kLayoutSW128);
-          umma_f16_ss(tmem + kTmemO, a, b, kIdPV, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(bar(KV_EMPTY + g % kStages));
-        umma_commit(bar(PV_DONE + (g & 1)));
-      }
-      __syncwarp();
-    };
-    while (ok && walk.next(sg)) {
-      if (!(ok = warp_wait(bar(Q_FULL), seg_i & 1, p.err))) break;
-      const int L = p.seqlens[sg.b];
-      const int n_t = sg.t1 - sg.t0;
-      int s_next = 0, pv_next = 0;
-      uint64_t t_idle = 0;
-      while (pv_next < n_t) {
-        // P . C first when its P is ready (it frees a stage and a P buffer);
-        // otherwise S for the next tile whose data and S buffer are ready
-        bool did = false;
-        if (pv_next < s_next) {
-          const int g = g0 + pv_next;
-          bool ready = false;
-          if (lane == 0) ready = mbar_test_nb(bar(P_FULL + (g & 1)), (g >> 1) & 1);
-          if (__shfl_sync(0xffffffffu, ready, 0)) {
-            if (!(ok = warp_wait(bar(P_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
-            issue_pv(g, pv_next == 0);
-            ++pv_next;
-            did = true;
+          if (!did && s_next < n_t) {
+            const int g = g0 + s_next;
+            bool ready = false;
+            if (lane == 0)
+              ready = mbar_test_nb_cluster(bar(KV_FULL + g % kStages), (g / kStages) & 1) &&
+                      mbar_test_nb_cluster(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1);
+            if (__shfl_sync(0xffffffffu, ready, 0)) {
+              if (!(ok = warp_wait<true>(bar(KV_FULL + g % kStages), (g / kStages) & 1, p.err) &&
+                         warp_wait<true>(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err)))
+                break;
+              issue_s(g, s_next == n_t - 1);
+              ++s_next;
+              did = true;
+            }
           }
-        }
-        if (!did && s_next < n_t) {
-          const int g = g0 + s_next;
-          bool ready = false;
-          if (lane == 0)
-            ready = mbar_test_nb(bar(KV_FULL + g % kStages), (g / kStages) & 1) &&
-                    mbar_test_nb(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1);
-          if (__shfl_sync(0xffffffffu, ready, 0)) {
-            if (!(ok = warp_wait(bar(KV_FULL + g % kStages), (g / kStages) & 1, p.err) &&
-                       warp_wait(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err)))
-              break;
-            issue_s(g, sg.t0 + s_next, L, s_next == n_t - 1);
-            ++s_next;
-            did = true;
+          if (did) {
+            t_idle = 0;
+          } else if (t_idle == 0) {
+            t_idle = globaltimer();
+          } else if (globaltimer() - t_idle > kWaitLimitNs) {
+            if (lane == 0) atomicOr(p.err, MLA_DEVFLAG_TIMEOUT);
+            ok = false;
+            break;
           }
         }
-        if (did) {
-          t_idle = 0;
-        } else if (t_idle == 0) {
-          t_idle = globaltimer();
-        } else if (globaltimer() - t_idle > kWaitLimitNs) {
-          if (lane == 0) atomicOr(p.err, MLA_DEVFLAG_TIMEOUT);
-          ok = false;
-          break;
-        }
+        g0 += n_t;
+        ++seg_i;
       }
-      g0 += n_t;
-      ++seg_i;
-    }
-    // every MMA issued by this thread has completed before TMEM is freed
-    if (lane == 0) {
-      umma_commit(bar(MMA_FINAL));
-      mbar_wait(bar(MMA_FINAL), 0, p.err, MLA_DEVFLAG_TIMEOUT);
-    }
-    __syncwarp();
-  } else if (warp == kWarpXchg) {
-    // ------------------------------------------------------------ exchange
-    // For every tile g in order: ship our staged partial S of tile g to the
-    // peer; then, once our softmax warps have read the peer's tile g, arm the
-    // receive barrier for tile g + 1 and tell the peer it may send again.
-    ChunkWalk walk;
-    walk.init(p.tile_prefix, p.B, chunk, cs);
-    Segment sg;
-    int total = 0;
-    while (walk.next(sg)) total += sg.t1 - sg.t0;
-    const uint32_t xin_peer = mapa(sbase + kOffXin, peer);
-    const uint32_t xfull_peer = mapa(bar(X_FULL), peer);
-    const uint32_t xempty_peer = mapa(bar(X_EMPTY), peer);
-    bool ok = true;
-    for (int g = 0; ok && g < total; ++g) {
-      if (!(ok = warp_wait(bar(X_OUT_READY), g & 1, p.err))) break;
-      if (!(ok = warp_wait<true>(bar(X_EMPTY), (g & 1) ^ 1, p.err))) break;  // peer read g - 1
+      // every MMA issued by this thread has completed before TMEM is freed
       if (lane == 0) {
-        bulk_copy_to_peer(xin_peer, sbase + kOffXout, kXBytes, xfull_peer);
-        bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(bar(X_OUT_FREE));
-      }
-      if (!(ok = warp_wait(bar(X_READ), g & 1, p.err))) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(X_FULL), kXBytes);  // tile g + 1
-        mbar_arrive_remote(xempty_peer);
+        umma_commit_pair(bar(MMA_FINAL), 1);
+        mbar_wait(bar(MMA_FINAL), 0, p.err, MLA_DEVFLAG_TIMEOUT);
       }
       __syncwarp();
     }
   } else if (warp >= kWarpSoftmax0) {
     // ------------------------------------------------------------ softmax
     const int sw_warp = warp - kWarpSoftmax0;       // 0..7
-    const int half = sw_warp >> 2;                  // tile columns [32 half, +32)
-    const int quad = warp & 3;                      // TMEM lanes [32 quad, +32)
-    const int row = quad * 32 + lane;               // head
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t sw = static_cast<uint32_t>(row & 7);
-    const uint32_t xout_row = sbase + kOffXout + row * 256;
-    const uint32_t xin_row = sbase + kOffXin + row * 256;
-    float* red = reinterpret_cast<float*>(base + kOffRed);  // [parity][half][row]
-    float* sums = reinterpret_cast<float*>(base + kOffSum); // [quantity][half][row]
+    const int c = sw_warp >> 2;                     // tokens [32c, 32c + 32) of a tile
+    const int qd = warp & 3;                        // TMEM lanes [32 qd, 32 qd + 32)
+    const int jh = lane >> 4;                       // S row half: partial over CTA jh's columns
+    const int hS = 16 * qd + (lane & 15);           // head (local) of this thread's S row
+    const int hO = (32 * qd + lane) & 63;           // head (local) of this thread's O lane
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+    const uint32_t sw = static_cast<uint32_t>(hS & 7);
+    float* red = reinterpret_cast<float*>(base + kOffRed);   // [parity][c][head]
+    float* sums = reinterpret_cast<float*>(base + kOffSum);  // [kind][c][head]
     const float c_log2 = p.scale_log2;
-    uint32_t pair_phase = 0;
-    // barrier between the two warps sharing these rows (bounded wait)
-    auto sync_pair = [&]() -> bool {
+    uint32_t grp_phase = 0;
+    auto rendezvous = [&]() -> bool {
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(SM_PAIR + quad));
-      return warp_wait(bar(SM_PAIR + quad), (pair_phase++) & 1, p.err);
-    };
-    // S_g (this thread's 32 columns) -> registers; free the S buffer; stage
-    // the row in the send buffer for the exchange warp.
-    auto fetch_and_stage = [&](int g, float (&dst)[32]) -> bool {
-      if (!warp_wait(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err)) return false;
-      tc_fence_after();
-      tmem_ld32(tmem + lane_base + kTmemS + (g & 1) * 64 + half * 32, dst);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(S_EMPTY + (g & 1)));
-      if (!warp_wait(bar(X_OUT_FREE), (g & 1) ^ 1, p.err)) return false;  // send of g - 1 left
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t chunk = static_cast<uint32_t>(half * 8 + k);
-        st_shared_v4(xout_row + ((chunk ^ sw) << 4), __float_as_uint(dst[4 * k]),
-                     __float_as_uint(dst[4 * k + 1]), __float_as_uint(dst[4 * k + 2]),
-                     __float_as_uint(dst[4 * k + 3]));
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(X_OUT_READY));
-      return true;
+      if (lane == 0) mbar_arrive(bar(GRP));
+      return warp_wait(bar(GRP), (grp_phase++) & 1, p.err);
     };
 
     ChunkWalk walk;
     walk.init(p.tile_prefix, p.B, chunk, cs);
     Segment sg;
-    int g = 0, seg_i = 0;
+    int g = 0;
     bool ok = true;
     while (ok && walk.next(sg)) {
       const int L = p.seqlens[sg.b];
       const int L_eff = L - p.s_q + 1 + qrow;  // positions this query row may see
       const int n_t = sg.t1 - sg.t0;
-
-      // ---- this segment's query: latent columns into TMEM, RoPE columns
-      // into shared memory (64-byte swizzle, the S operand layout)
-      if (seg_i > 0 && !(ok = warp_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err))) break;
-      {
-        const __nv_bfloat16* qrow_ptr =
-            row < p.n_h ? p.q + ((size_t)(sg.b * p.s_q + qrow) * p.n_h + row) * kWidth : nullptr;
-        uint32_t qw[32];
-        for (int part = 0; part < 2; ++part) {  // 2 x 64 latent values per thread
-          const uint4* src = qrow_ptr ? reinterpret_cast<const uint4*>(
-                                            qrow_ptr + rank * kLatPerCta + half * 128 + part * 64)
-                                      : nullptr;
+      // m_s: running max of the S head (weights); m_o: the same sequence of
+      // values for the O head (rescaling), derived from the same shared maxima
+      float m_s = -INFINITY, m_o = -INFINITY, l = 0.f, l_exact = 0.f;
+      for (int jt = 0; jt < n_t; ++jt, ++g) {
+        const int t = sg.t0 + jt;
+        // ---- partial scores of tile g -> registers; free the S buffer
+        if (!(ok = warp_wait<true>(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
+        tc_fence_after();
+        float own[32];
+        {
+          float va[32], vb[32];
+          const uint32_t sb = tmem + lane_base + kTmemS + (g & 1) * 128 + 32 * c;
+          tmem_ld32(sb, va);
+          tmem_ld32(sb + 64, vb);
+          tmem_wait_ld();
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 x = src ? src[v] : make_uint4(0, 0, 0, 0);
-            qw[4 * v] = x.x;
-            qw[4 * v + 1] = x.y;
-            qw[4 * v + 2] = x.z;
-            qw[4 * v + 3] = x.w;
-          }
-          tmem_st32u(tmem + lane_base + kTmemQ + half * 64 + part * 32, qw);
+          for (int k = 0; k < 32; ++k) own[k] = jh ? vb[k] : va[k];
         }
-        // RoPE: 32 values = 4 chunks of 16 B; half h writes chunks 2h, 2h + 1
-        const uint4* rsrc = qrow_ptr ? reinterpret_cast<const uint4*>(
-                                           qrow_ptr + kDc + rank * kRopePerCta)
-                                     : nullptr;
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const uint32_t c = static_cast<uint32_t>(half * 2 + v);
-          const uint4 x = rsrc ? rsrc[c] : make_uint4(0, 0, 0, 0);
-          st_shared_v4(sbase + kOffQRope + row * 64 + ((c ^ ((row >> 1) & 3)) << 4), x.x, x.y, x.z,
-                       x.w);
-        }
-        fence_proxy_async_smem();
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(Q_FULL));
-      }
-
-      float m = -INFINITY, l = 0.f, l_exact = 0.f;
-      float s[32], s_next[32];
-      if (!(ok = fetch_and_stage(g, s))) break;
-      for (int j = 0; j < n_t; ++j, ++g) {
-        const int t = sg.t0 + j;
-        // (1) the peer's partial of this tile; S = own + peer
-        if (!(ok = warp_wait<true>(bar(X_FULL), g & 1, p.err))) break;
+        if (lane == 0) mbar_arrive_remote(lead_bar(S_EMPTY + (g & 1)));
+        // S = partial(CTA 0 columns) + partial(CTA 1 columns): lane jh keeps
+        // tokens [16 jh, 16 jh + 16) of its 32 and hands the rest to lane ^ 16
+        float sc[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t chunk = static_cast<uint32_t>(half * 8 + k);
-          const float4 v = ld_shared_v4(xin_row + ((chunk ^ sw) << 4));
-          s[4 * k] += v.x;
-          s[4 * k + 1] += v.y;
-          s[4 * k + 2] += v.z;
-          s[4 * k + 3] += v.w;
+        for (int k = 0; k < 16; ++k) {
+          const float send = jh ? own[k] : own[16 + k];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+          sc[k] = (jh ? own[16 + k] : own[k]) + recv;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(X_READ));
-        // (2) stage the next tile's partial before this tile's arithmetic
-        if (j + 1 < n_t && !(ok = fetch_and_stage(g + 1, s_next))) break;
-
-        // (3) masked online softmax in log2 units
-        const int nv = L_eff - t * kTileTokens - half * 32;  // valid columns of this half
-        if (nv < 32) {
+        const int nv = L_eff - (t * kTileTokens + 32 * c + 16 * jh);  // valid of these 16
+        if (nv < 16) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c >= nv) s[c] = -INFINITY;
+          for (int k = 0; k < 16; ++k)
+            if (k >= nv) sc[k] = -INFINITY;
         }
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int k = 0; k < 16; k += 2) {
+          mx0 = fmaxf(mx0, sc[k]);
+          mx1 = fmaxf(mx1, sc[k + 1]);
         }
-        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-        red[((g & 1) * 2 + half) * 128 + row] = mx;
-        if (!(ok = sync_pair())) break;
-        mx = fmaxf(mx, red[((g & 1) * 2 + (half ^ 1)) * 128 + row]) * c_log2;  // scale > 0
-        const float m_new = fmaxf(m, mx);
-        const bool resc = m_new > m + kRescaleThreshold;
-        float alpha = 1.f;
-        if (resc) {
-          alpha = ex2_approx(m - m_new);
-          m = m_new;
+        float mx = fmaxf(mx0, mx1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (jh == 0) red[((g & 1) * 2 + c) * 64 + hS] = mx;
+        if (!(ok = rendezvous())) break;
+        // tile maximum (raw scores; scale > 0 commutes with max), the same
+        // expression for the S head and for the O head
+        const float* rd = red + (g & 1) * 2 * 64;
+        const float t_s = fmaxf(rd[hS], rd[64 + hS]) * c_log2;
+        const float t_o = fmaxf(rd[hO], rd[64 + hO]) * c_log2;
+        float alpha_s = 1.f, alpha_o = 1.f;
+        bool resc_o = false;
+        {
+          const float mn = fmaxf(m_s, t_s);
+          if (mn > m_s + kRescaleThreshold) {
+            alpha_s = ex2_approx(m_s - mn);
+            m_s = mn;
+          }
+          const float mo = fmaxf(m_o, t_o);
+          if (mo > m_o + kRescaleThreshold) {
+            alpha_o = ex2_approx(m_o - mo);
+            m_o = mo;
+            resc_o = true;
+          }
         }
-        const float neg_m = m == -INFINITY ? 0.f : -m;
+        const float neg_m = m_s == -INFINITY ? 0.f : -m_s;
         float r0 = 0.f, r1 = 0.f, e0 = 0.f, e1 = 0.f;
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float a = ex2_approx(fmaf(s[c], c_log2, neg_m));
-          const float b = ex2_approx(fmaf(s[c + 1], c_log2, neg_m));
+        for (int k = 0; k < 16; k += 2) {
+          const float a = ex2_approx(fmaf(sc[k], c_log2, neg_m));
+          const float b = ex2_approx(fmaf(sc[k + 1], c_log2, neg_m));
           const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
           const float2 pf = __bfloat1622float2(pr);
-          if (c & 2) { r1 += pf.x + pf.y; e1 += a + b; } else { r0 += pf.x + pf.y; e0 += a + b; }
-          pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&pr);
+          if (k & 2) { r1 += pf.x + pf.y; e1 += a + b; } else { r0 += pf.x + pf.y; e0 += a + b; }
+          pk[k >> 1] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         // u is normalised by the sum of the rounded weights it was built
         // from; lse uses the unrounded weights
-        l = l * alpha + (r0 + r1);
-        l_exact = l_exact * alpha + (e0 + e1);
+        l = l * alpha_s + (r0 + r1);
+        l_exact = l_exact * alpha_s + (e0 + e1);
 
         // P buffer g&1 was last read by PV_{g-2}; O may be rescaled only after
         // PV_{g-1} (tiles of an earlier segment were retired by that segment's
-        // epilogue)
-        if (j >= 2 && !(ok = warp_wait(bar(PV_DONE + (g & 1)), ((g - 2) >> 1) & 1, p.err))) break;
-        if (j >= 1 && __any_sync(0xffffffffu, resc)) {
-          if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
+        // epilogue, and the first P . C of a segment overwrites O)
+        if (jt >= 2 && !(ok = warp_wait<true>(bar(PV_DONE + (g & 1)), ((g - 2) >> 1) & 1, p.err)))
+          break;
+        if (jt >= 1 && __any_sync(0xffffffffu, resc_o)) {
+          if (!(ok = warp_wait<true>(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err)))
+            break;
           tc_fence_after();
           for (int c0 = 0; c0 < 128; c0 += 32) {
             float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + half * 128 + c0, o);
+            tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tmem + lane_base + kTmemO + half * 128 + c0, o);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha_o;
+            tmem_st32(tmem + lane_base + kTmemO + c * 128 + c0, o);
           }
           tmem_wait_st();
         }
-        // P row (64 tokens = 128 B, 128-byte swizzle); this thread writes
-        // its half: 16-byte chunks 4h .. 4h + 3
-        const uint32_t prow = sbase + kOffP + (g & 1) * kPBytes + row * 128;
+        // P row hS (64 tokens = 128 B, 128-byte swizzle); this thread writes
+        // tokens [32c + 16jh, +16): 16-byte chunks 4c + 2jh and 4c + 2jh + 1
+        const uint32_t prow = sbase + kOffP + (g & 1) * kPBytes + hS * 128;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t c = static_cast<uint32_t>(half * 4 + k);
-          st_shared_v4(prow + ((c ^ sw) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t ch = static_cast<uint32_t>(4 * c + 2 * jh + k);
+          st_shared_v4(prow + ((ch ^ sw) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
+                       pk[4 * k + 3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(P_FULL + (g & 1)));
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[c] = s_next[c];
+        if (lane == 0) mbar_arrive_remote(lead_bar(P_FULL + (g & 1)));
       }
       if (!ok) break;
 
-      // ---- epilogue: u = O / l (this thread's 128 of the CTA's 256 columns)
-      sums[(0 * 2 + half) * 128 + row] = l;
-      sums[(1 * 2 + half) * 128 + row] = l_exact;
-      if (!(ok = sync_pair())) break;
-      l += sums[(0 * 2 + (half ^ 1)) * 128 + row];
-      l_exact += sums[(1 * 2 + (half ^ 1)) * 128 + row];
-      if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse = l_exact > 0.f ? (m + log2f(l_exact)) * 0.69314718055994531f : -INFINITY;
-      const bool write = row < p.n_h;
-      const size_t orow = (size_t)(sg.b * p.s_q + qrow) * p.n_h + row;
-      const size_t slot = sg.whole ? 0 : (size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow;
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + kTmemO + half * 128 + c0, o);
-        tmem_wait_ld();
-        if (!write) continue;
-        const int col = rank * kLatPerCta + half * 128 + c0;
-        if (sg.whole) {
-          uint4* dst = reinterpret_cast<uint4*>(p.u + orow * kDc + col);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 h2 =
-                  __floats2bfloat162_rn(o[8 * v + 2 * e] * inv, o[8 * v + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.part_u + (slot * p.n_h + row) * kDc + col);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(o[4 * v] * inv, o[4 * v + 1] * inv, o[4 * v + 2] * inv,
-                                 o[4 * v + 3] * inv);
+      // ---- epilogue: u = O / l for this thread's O lane (one head, 128
+      // consecutive latent columns)
+      {
+        const float l2 = l + __shfl_xor_sync(0xffffffffu, l, 16);
+        const float e2 = l_exact + __shfl_xor_sync(0xffffffffu, l_exact, 16);
+        if (jh == 0) {
+          sums[(0 * 2 + c) * 64 + hS] = l2;
+          sums[(1 * 2 + c) * 64 + hS] = e2;
         }
       }
-      if (write && rank == 0 && half == 0) {
+      if (!(ok = rendezvous())) break;
+      const float l_o = sums[(0 * 2 + 0) * 64 + hO] + sums[(0 * 2 + 1) * 64 + hO];
+      const float le_o = sums[(1 * 2 + 0) * 64 + hO] + sums[(1 * 2 + 1) * 64 + hO];
+      if (!(ok = warp_wait<true>(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
+      tc_fence_after();
+      const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
+      const size_t row0 = (size_t)(sg.b * p.s_q + qrow) * p.n_h;
+      const size_t slot = sg.whole ? 0 : (size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow;
+      const int col0 = 256 * c + 128 * (qd >> 1);  // latent column of TMEM column kTmemO + 128c
+      // rows leave through a 2 KB per-warp staging area (the P buffers are
+      // free now) so that each global store instruction writes 64 contiguous
+      // bytes of 8 rows; 16-byte chunks are rotated by (row >> 1) & 3 so that
+      // neither side of the staging has bank conflicts
+      const uint32_t stg = sbase + kOffP + sw_warp * 2048;
+      const uint32_t my_row = stg + lane * 64;
+      const uint32_t my_rot = static_cast<uint32_t>((lane >> 1) & 3);
+      auto flush = [&](int col_first, bool as_bf16) {
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = (lane >> 2) + 8 * k, ch = lane & 3;
+          const float4 v = ld_shared_v4(stg + r * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
+          const int head = 64 * (int)rank + ((32 * qd + r) & 63);
+          if (head < p.n_h) {
+            if (as_bf16)
+              *reinterpret_cast<float4*>(p.u + (row0 + head) * kDc + col_first + 8 * ch) = v;
+            else
+              *reinterpret_cast<float4*>(p.part_u + (slot * p.n_h + head) * kDc + col_first +
+                                         4 * ch) = v;
+          }
+        }
+        __syncwarp();
+      };
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
+        tmem_wait_ld();
         if (sg.whole) {
-          if (p.lse != nullptr) p.lse[orow] = lse;
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * e] * inv, o[2 * e + 1] * inv);
+            w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(my_row + ((k ^ my_rot) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
+                         w[4 * k + 3]);
+          flush(col0 + c0, true);
         } else {
-          p.part_lse[slot * p.n_h + row] = lse;
+          for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float* v = o + 16 * hf + 4 * k;
+              st_shared_v4(my_row + ((k ^ my_rot) << 4), __float_as_uint(v[0] * inv),
+                           __float_as_uint(v[1] * inv), __float_as_uint(v[2] * inv),
+                           __float_as_uint(v[3] * inv));
+            }
+            flush(col0 + c0 + 16 * hf, false);
+          }
+        }
+      }
+      const int head = 64 * (int)rank + hO;
+      if (head < p.n_h && qd < 2 && c == 0) {
+        const float lse = le_o > 0.f ? (m_o + log2f(le_o)) * 0.69314718055994531f : -INFINITY;
+        if (sg.whole) {
+          if (p.lse != nullptr) p.lse[row0 + head] = lse;
+        } else {
+          p.part_lse[slot * p.n_h + head] = lse;
         }
       }
       tc_fence_before();
-      ++seg_i;
     }
   }
 
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // all paired MMAs are complete and no arrival is still on its way
   if (warp == kWarpAlloc) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
-  cluster_sync();  // no CTA leaves while its peer may still send into its shared memory
+  cluster_sync();
 }
 
 }  // namespace
@@ -674,7 +701,6 @@ int decode_sm100_prepare() {
 cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s) {
   Params p;
   p.maps = maps;
-  p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.block_table = a.block_table;
   p.seqlens = a.seqlens;
   p.header = a.header;

@@ -46,10 +46,13 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s);
 
 // Tensor-core decode for n_h <= 128, d_c = 512, d_R = 64, bf16.
-// maps over the cache [rows, 576]: latent boxes 64 x 64 (128-byte swizzle),
-// RoPE boxes 32 x 64 (64-byte swizzle).
+// kv maps over the cache [rows, 576]: latent boxes 64 x 64 rows (128-byte
+// swizzle), RoPE boxes 32 x 64 rows (64-byte swizzle).  q maps over the
+// queries [B * s_q, n_h, 576]: latent boxes 64 x 16 heads x 1 (128-byte
+// swizzle), RoPE boxes 32 x 16 heads x 1 (64-byte swizzle); heads past n_h
+// read as zero.
 struct Sm100Maps {
-  CUtensorMap kv_lat, kv_rope;
+  CUtensorMap kv_lat, kv_rope, q_lat, q_rope;
 };
 cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s);
 size_t decode_sm100_smem_bytes();
