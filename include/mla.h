@@ -59,6 +59,7 @@ typedef enum { MLA_DTYPE_BF16 = 0, MLA_DTYPE_FP32 = 1 } mla_dtype;
 #define MLA_DEVFLAG_BAD_SEQLEN 0x1  /* seqlens[b] < s_q or > max_pages_per_seq*page_size */
 #define MLA_DEVFLAG_BAD_PAGE 0x2    /* block_table entry outside [0, num_pages) */
 #define MLA_DEVFLAG_TIMEOUT 0x4     /* a device-side wait gave up (kernel returned early) */
+#define MLA_DEVFLAG_LAYOUT 0x8      /* a kernel's shared memory was not 1024-byte aligned (it returned at once) */
 
 const char* mla_status_string(mla_status s);
 

@@ -166,6 +166,7 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   a.scale = p->softmax_scale;
   a.bf16 = p->dtype == MLA_DTYPE_BF16;
   r->tc = use_tensor_cores(p, r->dev);
+  a.part_bf16 = r->tc;
   return MLA_OK;
 }
 

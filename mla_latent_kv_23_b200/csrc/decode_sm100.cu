@@ -35,7 +35,10 @@
 //
 // TMEM per CTA (512 columns): S 2 x 128 (double-buffered) | O 256.
 // Shared memory per CTA: Q (128 rows x 288 values, the S operand A) 72 KB;
-// 3 tile stages of 36 KB; two P buffers (64 heads x 64 tokens bf16) of 8 KB.
+// 4 tile stages of 36 KB; P (64 heads x 64 tokens bf16) as two 32-token
+// halves with 64-byte swizzle: tokens 0-31 in the tile's own RoPE block (free
+// once S of the tile is done, and held until its P . C releases the stage),
+// tokens 32-63 in a two-slot 4 KB ring.
 // One shared-memory copy of a tile serves both contractions: a TMA load with
 // 128-byte swizzle writes each 64-column block as 64 rows x 128 B, the
 // K-major layout of the S operand and the MN-major layout of the P . C
@@ -43,16 +46,15 @@
 //
 // Roles (384 threads): warp 0 = TMA producer for this CTA's columns (the
 // whole warp prefetches block-table entries, lane 0 issues copies); warp 1 =
-// MMA issuer (even CTA only): S for whichever tile is ready (up to two tiles
-// ahead), P . C as soon as P is ready; warp 2 = TMEM allocator; warp 3 =
-// relay: loads the segment's query by TMA, zeroes cache rows past a
-// sequence's end in this CTA's stage, and signals the even CTA's barriers
-// that this CTA's operands are in place; warps 4-11 = softmax: warp 4 + 4c + q
-// reads TMEM lanes [32q, 32q + 32) and tokens [32c, 32c + 32) of a tile.
-// Each thread finishes 16 scores of one head; the row maximum is shared
-// through shared memory with one 8-warp rendezvous per tile.  O rows are
-// rescaled by the warp that can reach their TMEM lanes, which derives the
-// same maximum from the same shared values.
+// S issuer (even CTA only); warp 2 = TMEM allocator, then P . C issuer
+// (even CTA only); warp 3 = relay: loads the segment's query by TMA,
+// zeroes cache rows past a sequence's end in this CTA's stage, and signals
+// the even CTA's barriers that this CTA's operands are in place; warps 4-11
+// = softmax: warp 4 + 4c + q reads TMEM lanes [32q, 32q + 32) and tokens
+// [32c, 32c + 32) of a tile.  Each thread finishes 16 scores of one head; the
+// row maximum is shared through shared memory with one 8-warp rendezvous per
+// tile.  O rows are rescaled by the warp that can reach their TMEM lanes,
+// which derives the same maximum from the same shared values.
 //
 // Work: the plan stage cuts the batch's tiles into equal chunks; cluster c
 // handles chunk c / s_q for query row c % s_q, walking its segments in order.
@@ -69,7 +71,7 @@ using namespace ptx;
 
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpAlloc = 2, kWarpRelay = 3, kWarpSoftmax0 = 4;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kDc = 512;
 
 constexpr uint32_t kKvBlk = 64 * 128;                    // tile: 64 rows x 64 cols, SW128
@@ -78,33 +80,39 @@ constexpr uint32_t kStageBytes = 4 * kKvBlk + kKvRope;   // 36864
 constexpr uint32_t kQBlk = 128 * 128;                    // Q: 128 rows x 64 cols, SW128
 constexpr uint32_t kQRope = 128 * 64;                    // Q: 128 rows x 32 cols, SW64
 constexpr uint32_t kQBytes = 4 * kQBlk + kQRope;         // 73728
-constexpr uint32_t kPBytes = 64 * 128;                   // 64 heads x 64 tokens bf16, SW128
+constexpr uint32_t kPHalf = 64 * 64;                     // 64 heads x 32 tokens bf16, SW64
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKv = kOffQ + kQBytes;
-constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;   // [2]
-constexpr uint32_t kOffRed = kOffP + 2 * kPBytes;            // float [2 parity][2 c][64 heads]
+constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;   // [2] second halves of P
+constexpr uint32_t kOffRed = kOffP + 2 * kPHalf;             // float [2 parity][2 c][64 heads]
 constexpr uint32_t kOffSum = kOffRed + 2 * 2 * 64 * 4;       // float [2 kind][2 c][64 heads]
-constexpr uint32_t kOffBar = kOffSum + 2 * 2 * 64 * 4;
+constexpr uint32_t kOffScratch = kOffSum + 2 * 2 * 64 * 4;    // 16 words written by the odd CTA's signals
+constexpr uint32_t kOffBar = kOffScratch + 64;
 
+// Barriers of the even CTA that the odd CTA signals ("paired" below) count
+// the even CTA's own arrivals, and the odd CTA's signals as 4-byte
+// transactions (st.async) that one of the even CTA's arrivals announces.
 enum Bar {
-  LOCAL_FULL = 0,                  // [3] this CTA's TMA bytes of a stage
-  KV_FULL = LOCAL_FULL + kStages,  // [3] even CTA: both CTAs' stage ready (2 relay arrivals)
-  KV_EMPTY = KV_FULL + kStages,    // [3] P . C of the stage's tile done (paired commit)
+  LOCAL_FULL = 0,                  // [stage] this CTA's TMA bytes of a stage (tail tiles)
+  KV_FULL = LOCAL_FULL + kStages,  // [stage] even CTA: both CTAs' stage ready; full tiles count
+                                   //     both CTAs' TMA bytes, tail tiles the relays' signals
+  KV_EMPTY = KV_FULL + kStages,    // [stage] P . C of the stage's tile done (paired commit)
   S_FULL = KV_EMPTY + kStages,     // [2] per S buffer (paired commit)
-  S_EMPTY = S_FULL + 2,            // [2] even CTA: 16 softmax warps read the S buffer
-  P_FULL = S_EMPTY + 2,            // [2] even CTA: 16 softmax warps wrote P
+  S_EMPTY = S_FULL + 2,            // [2] even CTA, paired: softmax warps read the S buffer
+  P_FULL = S_EMPTY + 2,            // [2] even CTA, paired: softmax warps wrote P
   PV_DONE = P_FULL + 2,            // [2] (paired commit)
   Q_LOCAL = PV_DONE + 2,           // this CTA's query bytes
-  Q_FULL,                          // even CTA: both queries in place (2 relay arrivals)
+  Q_FULL,                          // even CTA, paired: both queries in place (relays)
   Q_EMPTY,                         // last S of a segment done (paired commit)
   GRP,                             // the 8 softmax warps of this CTA
-  MMA_FINAL,
+  MMA_FINAL,                       // even CTA: all S issued so far are complete
+  MMA_FINAL_PV,                    // even CTA: all P . C issued so far are complete
   BAR_COUNT
 };
 constexpr uint32_t kOffTmemSlot = kOffBar + BAR_COUNT * 8;
 constexpr uint32_t kSmemUsed = kOffTmemSlot + 16;
-constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
+constexpr size_t kSmemBytes = kSmemUsed;  // the base is 1024-byte aligned (checked at entry)
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;     // 2 x 128 columns
@@ -128,7 +136,7 @@ struct Params {
   const int* header;
   const int* tile_prefix;
   const int* split_base;
-  float* part_u;
+  __nv_bfloat16* part_u;  // split partials of u, bf16
   float* part_lse;
   __nv_bfloat16* u;
   float* lse;
@@ -137,45 +145,82 @@ struct Params {
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-// Every lane of the warp polls; the warp agrees on the outcome.
+// Lane 0 polls (a warp of spinning lanes only adds shared-memory traffic);
+// the shuffle hands the outcome, and the ordering, to the rest of the warp.
 template <bool kCluster = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err) {
-  const bool ok = mbar_wait<kCluster>(bar, parity, err, MLA_DEVFLAG_TIMEOUT);
-  return __all_sync(0xffffffffu, ok);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(bar, parity, err, MLA_DEVFLAG_TIMEOUT);
+  return __shfl_sync(0xffffffffu, ok, 0);
+}
+
+// Both phases complete; the two tests of each poll are independent, so their
+// shared-memory latencies overlap.
+__device__ __forceinline__ bool warp_wait2(uint32_t bar0, uint32_t par0, uint32_t bar1,
+                                           uint32_t par1, int* err) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    const uint64_t t0 = cycles();
+    uint32_t n = 0;
+    while (!(mbar_test_nb(bar0, par0) & mbar_test_nb(bar1, par1))) {
+      if ((++n & 31u) == 0 && cycles() - t0 > kWaitLimitCycles) {
+        atomicOr(err, MLA_DEVFLAG_TIMEOUT);
+        ok = false;
+        break;
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok, 0);
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_sm100_kernel(const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
-  uint8_t* base = smem_raw + (sbase - raw_addr);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  uint8_t* base = smem_raw;
+  if (sbase & 1023u) {  // the swizzled layouts need it; nothing has been started yet
+    if (threadIdx.x == 0) atomicOr(p.err, MLA_DEVFLAG_LAYOUT);
+    return;
+  }
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cid = blockIdx.x >> 1;
   const int chunk = cid / p.s_q, qrow = cid % p.s_q;
   auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * i; };
-  // barriers that live in the even CTA, addressed from either CTA
-  auto lead_bar = [&](int i) -> uint32_t { return mapa(bar(i), 0); };
+  // Signal a paired barrier of the even CTA: from the even CTA a local
+  // arrival (with `announce`, the one arrival per phase that also expects the
+  // odd CTA's `odd_bytes` of signals); from the odd CTA a non-blocking 4-byte
+  // st.async into scratch word `scratch_word` of the even CTA.
+  auto signal_lead = [&](int i, bool announce, uint32_t odd_bytes, int scratch_word) {
+    if (leader) {
+      if (announce)
+        mbar_arrive_expect_tx(bar(i), odd_bytes);
+      else
+        mbar_arrive(bar(i));
+    } else {
+      st_async_b32(mapa(sbase + kOffScratch + 4u * scratch_word, 0), 0u, mapa(bar(i), 0));
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(LOCAL_FULL + s), 1);
-      mbar_init(bar(KV_FULL + s), 2);
+      mbar_init(bar(KV_FULL + s), 1);
       mbar_init(bar(KV_EMPTY + s), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(S_FULL + i), 1);
-      mbar_init(bar(S_EMPTY + i), 16);
-      mbar_init(bar(P_FULL + i), 16);
+      mbar_init(bar(S_EMPTY + i), 8);
+      mbar_init(bar(P_FULL + i), 8);
       mbar_init(bar(PV_DONE + i), 1);
     }
     mbar_init(bar(Q_LOCAL), 1);
-    mbar_init(bar(Q_FULL), 2);
+    mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(Q_EMPTY), 1);
     mbar_init(bar(GRP), 8);
     mbar_init(bar(MMA_FINAL), 1);
+    mbar_init(bar(MMA_FINAL_PV), 1);
     fence_mbar_init();
   }
   if (warp == kWarpAlloc) {
@@ -206,11 +251,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     walk.init(p.tile_prefix, p.B, chunk, cs);
     Segment sg;
     int g = 0;
-    int last_n[kStages];
-    for (int s = 0; s < kStages; ++s) last_n[s] = -1;
+    int last_n[kStages], tail_n[kStages];  // uses of LOCAL_FULL per stage
+    for (int s = 0; s < kStages; ++s) last_n[s] = -1, tail_n[s] = 0;
     bool ok = true;
     while (ok && walk.next(sg)) {
       const int* bt = p.block_table + (size_t)sg.b * p.max_pages;
+      const int L = p.seqlens[sg.b];
       for (int t0 = sg.t0; ok && t0 < sg.t1; t0 += 32) {
         // each lane fetches the page of one upcoming tile
         int my_page = 0;
@@ -226,18 +272,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int page = __shfl_sync(0xffffffffu, my_page, i);
           if (lane == 0) {
             const int s = g % kStages, n = g / kStages;
-            ok = mbar_wait<true>(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT);
+            ok = mbar_wait(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT);
             if (ok) {
               const int tok = (t0 + i) * kTileTokens;
               const int y = page * p.page_size + tok % p.page_size;
               const uint32_t st = sbase + kOffKv + s * kStageBytes;
-              mbar_arrive_expect_tx(bar(LOCAL_FULL + s), kStageBytes);
-              for (int kc = 0; kc < 4; ++kc)
-                tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(LOCAL_FULL + s),
-                            lat_col(kc, (int)rank), y);
-              tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(LOCAL_FULL + s),
-                          kDc + 32 * (int)rank, y);
-              last_n[s] = n;
+              if (L - tok < kTileTokens) {
+                // tail tile: this CTA's relay zeroes the rows past the end
+                // once they land, then signals the even CTA
+                mbar_arrive_expect_tx(bar(LOCAL_FULL + s), kStageBytes);
+                for (int kc = 0; kc < 4; ++kc)
+                  tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(LOCAL_FULL + s),
+                              lat_col(kc, (int)rank), y);
+                tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(LOCAL_FULL + s),
+                            kDc + 32 * (int)rank, y);
+                last_n[s] = tail_n[s]++;
+              } else if (leader) {
+                // full tile: both CTAs' bytes complete on the even CTA's barrier
+                mbar_arrive_expect_tx(bar(KV_FULL + s), 2 * kStageBytes);
+                for (int kc = 0; kc < 4; ++kc)
+                  tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
+                              lat_col(kc, 0), y);
+                tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(KV_FULL + s), kDc, y);
+              } else {
+                const uint32_t full = mapa(bar(KV_FULL + s), 0);
+                for (int kc = 0; kc < 4; ++kc)
+                  tma_load_2d_to_pair(st + kc * kKvBlk, &p.maps.kv_lat, full, lat_col(kc, 1), y);
+                tma_load_2d_to_pair(st + 4 * kKvBlk, &p.maps.kv_rope, full, kDc + 32, y);
+              }
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -245,7 +307,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // wait for this thread's own copies in flight before the CTA may exit
+    // wait for this thread's tail copies in flight before the CTA may exit
+    // (full tiles are consumed by the paired MMAs before the final cluster
+    // barrier)
     if (lane == 0)
       for (int s = 0; s < kStages; ++s)
         if (last_n[s] >= 0) mbar_wait(bar(LOCAL_FULL + s), last_n[s] & 1, p.err, MLA_DEVFLAG_TIMEOUT);
@@ -256,13 +320,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     walk.init(p.tile_prefix, p.B, chunk, cs);
     Segment sg;
     int g = 0, seg_i = 0;
+    int tail_n[kStages];  // uses of LOCAL_FULL per stage, in tile order
+    for (int s = 0; s < kStages; ++s) tail_n[s] = 0;
     bool ok = true;
     bool q_in_flight = false;
     while (ok && walk.next(sg)) {
       // this segment's query rows (h, j) = Q[64 rank + 16 qd + i, columns of
       // CTA j], stored as row 32 qd + 16 j + i; heads >= n_h read as zero
       // (the tensor map ends there)
-      if (seg_i > 0 && !(ok = warp_wait<true>(bar(Q_EMPTY), (seg_i - 1) & 1, p.err))) break;
+      if (seg_i > 0 && !(ok = warp_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err))) break;
       if (lane == 0) {
         const int z = sg.b * p.s_q + qrow;
         mbar_arrive_expect_tx(bar(Q_LOCAL), kQBytes);
@@ -280,31 +346,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       q_in_flight = true;
       if (!(ok = warp_wait(bar(Q_LOCAL), seg_i & 1, p.err))) break;
       q_in_flight = false;
-      if (lane == 0) mbar_arrive_remote(lead_bar(Q_FULL));
+      if (lane == 0) signal_lead(Q_FULL, true, 4u, 8);
       __syncwarp();
 
       const int L = p.seqlens[sg.b];
       for (int t = sg.t0; t < sg.t1; ++t, ++g) {
         const int s = g % kStages;
-        if (!(ok = warp_wait(bar(LOCAL_FULL + s), (g / kStages) & 1, p.err))) break;
         const int rows_valid = L - t * kTileTokens;
-        if (rows_valid < kTileTokens) {
-          // rows past the sequence end may hold anything; make them zero so
-          // that 0-probability x garbage cannot turn into NaN in P . C
-          uint8_t* tile = base + kOffKv + s * kStageBytes;
-          for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
-            if (lane < 8)
-              for (int kb = 0; kb < 4; ++kb)
-                *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
-                    make_uint4(0, 0, 0, 0);
-            if (lane < 4)
-              *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
+        if (rows_valid >= kTileTokens) continue;  // full tile: no relay
+        if (!(ok = warp_wait(bar(LOCAL_FULL + s), (tail_n[s]++) & 1, p.err))) break;
+        // rows past the sequence end may hold anything; make them zero so
+        // that 0-probability x garbage cannot turn into NaN in P . C
+        uint8_t* tile = base + kOffKv + s * kStageBytes;
+        for (int r = max(rows_valid, 0); r < kTileTokens; ++r) {
+          if (lane < 8)
+            for (int kb = 0; kb < 4; ++kb)
+              *reinterpret_cast<uint4*>(tile + kb * kKvBlk + r * 128 + lane * 16) =
                   make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
+          if (lane < 4)
+            *reinterpret_cast<uint4*>(tile + 4 * kKvBlk + r * 64 + lane * 16) =
+                make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead_bar(KV_FULL + s));
+        if (lane == 0) signal_lead(KV_FULL + s, true, 4u, 9);
         __syncwarp();
       }
       ++seg_i;
@@ -312,8 +377,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // a query copy still in flight must land before the CTA may exit
     if (q_in_flight && lane == 0) mbar_wait(bar(Q_LOCAL), seg_i & 1, p.err, MLA_DEVFLAG_TIMEOUT);
     __syncwarp();
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kWarpMma || warp == kWarpAlloc) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues every S, warp 2 (done allocating) every P . C.  The two
+    // streams touch disjoint TMEM and shared memory, and each commit tracks
+    // only its own thread's MMAs, so a P . C whose P is ready never waits
+    // behind an S being issued (issuing blocks while the tensor pipe's queue
+    // is full) and vice versa.
     if (leader) {
       constexpr uint32_t kIdS = idesc_bf16(256, 128, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, 256, true);
@@ -352,10 +422,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (lane == 0) {
           const uint32_t st = sbase + kOffKv + (g % kStages) * kStageBytes;
-          const uint32_t pa = sbase + kOffP + (g & 1) * kPBytes;
+          // P tokens 0-31 sit in the stage's RoPE block (S is done with it),
+          // tokens 32-63 in the second-half ring
+          const uint32_t pa0 = st + 4 * kKvBlk, pa1 = sbase + kOffP + (g & 1) * kPHalf;
           for (int blk = 0; blk < 2; ++blk)
             for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
-              const uint64_t a = smem_desc(pa + kk * 32, 16, 1024, kLayoutSW128);
+              const uint64_t a = smem_desc((kk < 2 ? pa0 : pa1) + (kk & 1) * 32, 16, 512, kLayoutSW64);
               const uint64_t b =
                   smem_desc(st + 2 * blk * kKvBlk + kk * 2048, kKvBlk, 1024, kLayoutSW128);
               umma_f16_ss_pair(tmem + kTmemO + blk * 128, a, b, kIdPV,
@@ -366,58 +438,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
+      // Fixed order per segment: S0 S1 S2, then P.C(j) S(j+3) for every tile
+      // j, so S runs two tiles ahead of P.C and the softmax of tile j has
+      // two S groups of tensor work to hide behind.  Each step polls only the
+      // barriers it needs (a barrier test costs ~150 cycles; re-testing a
+      // ready barrier is not free).
+      const bool s_issuer = warp == kWarpMma;
       while (ok && walk.next(sg)) {
-        if (!(ok = warp_wait<true>(bar(Q_FULL), seg_i & 1, p.err))) break;
         const int n_t = sg.t1 - sg.t0;
-        int s_next = 0, pv_next = 0;
-        uint64_t t_idle = 0;
-        while (pv_next < n_t) {
-          // P . C first when its P is ready (it frees a stage and a P buffer);
-          // otherwise S for the next tile whose data and S buffer are ready
-          bool did = false;
-          if (pv_next < s_next) {
-            const int g = g0 + pv_next;
-            bool ready = false;
-            if (lane == 0) ready = mbar_test_nb_cluster(bar(P_FULL + (g & 1)), (g >> 1) & 1);
-            if (__shfl_sync(0xffffffffu, ready, 0)) {
-              if (!(ok = warp_wait<true>(bar(P_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
-              issue_pv(g, pv_next == 0);
-              ++pv_next;
-              did = true;
-            }
+        if (s_issuer) {
+          // S(g) once its stage is loaded and its S buffer has been read
+          if (!(ok = warp_wait(bar(Q_FULL), seg_i & 1, p.err))) break;
+          for (int j = 0; ok && j < n_t; ++j) {
+            const int g = g0 + j;
+            if (!(ok = warp_wait2(bar(KV_FULL + g % kStages), (g / kStages) & 1,
+                                  bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err)))
+              break;
+            issue_s(g, j == n_t - 1);
           }
-          if (!did && s_next < n_t) {
-            const int g = g0 + s_next;
-            bool ready = false;
-            if (lane == 0)
-              ready = mbar_test_nb_cluster(bar(KV_FULL + g % kStages), (g / kStages) & 1) &&
-                      mbar_test_nb_cluster(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1);
-            if (__shfl_sync(0xffffffffu, ready, 0)) {
-              if (!(ok = warp_wait<true>(bar(KV_FULL + g % kStages), (g / kStages) & 1, p.err) &&
-                         warp_wait<true>(bar(S_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1, p.err)))
-                break;
-              issue_s(g, s_next == n_t - 1);
-              ++s_next;
-              did = true;
-            }
-          }
-          if (did) {
-            t_idle = 0;
-          } else if (t_idle == 0) {
-            t_idle = globaltimer();
-          } else if (globaltimer() - t_idle > kWaitLimitNs) {
-            if (lane == 0) atomicOr(p.err, MLA_DEVFLAG_TIMEOUT);
-            ok = false;
-            break;
+        } else {
+          // P . C(g) once P(g) is written
+          for (int j = 0; ok && j < n_t; ++j) {
+            const int g = g0 + j;
+            if (!(ok = warp_wait(bar(P_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
+            issue_pv(g, j == 0);
           }
         }
         g0 += n_t;
         ++seg_i;
       }
       // every MMA issued by this thread has completed before TMEM is freed
+      const int fin = s_issuer ? MMA_FINAL : MMA_FINAL_PV;
       if (lane == 0) {
-        umma_commit_pair(bar(MMA_FINAL), 1);
-        mbar_wait(bar(MMA_FINAL), 0, p.err, MLA_DEVFLAG_TIMEOUT);
+        umma_commit_pair(bar(fin), 1);
+        mbar_wait(bar(fin), 0, p.err, MLA_DEVFLAG_TIMEOUT);
       }
       __syncwarp();
     }
@@ -430,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int hS = 16 * qd + (lane & 15);           // head (local) of this thread's S row
     const int hO = (32 * qd + lane) & 63;           // head (local) of this thread's O lane
     const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-    const uint32_t sw = static_cast<uint32_t>(hS & 7);
+    const uint32_t sw64 = static_cast<uint32_t>((hS >> 1) & 3);  // 64-byte swizzle of row hS
     float* red = reinterpret_cast<float*>(base + kOffRed);   // [parity][c][head]
     float* sums = reinterpret_cast<float*>(base + kOffSum);  // [kind][c][head]
     const float c_log2 = p.scale_log2;
@@ -456,7 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int jt = 0; jt < n_t; ++jt, ++g) {
         const int t = sg.t0 + jt;
         // ---- partial scores of tile g -> registers; free the S buffer
-        if (!(ok = warp_wait<true>(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
+        if (!(ok = warp_wait(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
         tc_fence_after();
         float own[32];
         {
@@ -470,7 +524,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead_bar(S_EMPTY + (g & 1)));
+        if (lane == 0) signal_lead(S_EMPTY + (g & 1), sw_warp == 0, 32u, sw_warp);
         // S = partial(CTA 0 columns) + partial(CTA 1 columns): lane jh keeps
         // tokens [16 jh, 16 jh + 16) of its 32 and hands the rest to lane ^ 16
         float sc[16];
@@ -533,13 +587,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         l = l * alpha_s + (r0 + r1);
         l_exact = l_exact * alpha_s + (e0 + e1);
 
-        // P buffer g&1 was last read by PV_{g-2}; O may be rescaled only after
-        // PV_{g-1} (tiles of an earlier segment were retired by that segment's
-        // epilogue, and the first P . C of a segment overwrites O)
-        if (jt >= 2 && !(ok = warp_wait<true>(bar(PV_DONE + (g & 1)), ((g - 2) >> 1) & 1, p.err)))
+        // P's second-half slot g&1 was last read by PV_{g-2}; O may be
+        // rescaled only after PV_{g-1} (tiles of an earlier segment were
+        // retired by that segment's epilogue, and the first P . C of a segment
+        // overwrites O)
+        if (jt >= 2 && !(ok = warp_wait(bar(PV_DONE + (g & 1)), ((g - 2) >> 1) & 1, p.err)))
           break;
         if (jt >= 1 && __any_sync(0xffffffffu, resc_o)) {
-          if (!(ok = warp_wait<true>(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err)))
+          if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err)))
             break;
           tc_fence_after();
           for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -552,19 +607,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
         }
-        // P row hS (64 tokens = 128 B, 128-byte swizzle); this thread writes
-        // tokens [32c + 16jh, +16): 16-byte chunks 4c + 2jh and 4c + 2jh + 1
-        const uint32_t prow = sbase + kOffP + (g & 1) * kPBytes + hS * 128;
+        // P row hS, tokens [32c + 16jh, +16): half c of the row (32 tokens =
+        // 64 B, 64-byte swizzle) lives in the stage's RoPE block (c = 0) or
+        // in second-half slot g&1 (c = 1); 16-byte chunks 2jh and 2jh + 1
+        const uint32_t prow =
+            (c == 0 ? sbase + kOffKv + (g % kStages) * kStageBytes + 4 * kKvBlk
+                    : sbase + kOffP + (g & 1) * kPHalf) + hS * 64;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const uint32_t ch = static_cast<uint32_t>(4 * c + 2 * jh + k);
-          st_shared_v4(prow + ((ch ^ sw) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
+          const uint32_t ch = static_cast<uint32_t>(2 * jh + k);
+          st_shared_v4(prow + ((ch ^ sw64) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
                        pk[4 * k + 3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead_bar(P_FULL + (g & 1)));
+        if (lane == 0) signal_lead(P_FULL + (g & 1), sw_warp == 0, 32u, sw_warp);
       }
       if (!ok) break;
 
@@ -581,63 +639,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!(ok = rendezvous())) break;
       const float l_o = sums[(0 * 2 + 0) * 64 + hO] + sums[(0 * 2 + 1) * 64 + hO];
       const float le_o = sums[(1 * 2 + 0) * 64 + hO] + sums[(1 * 2 + 1) * 64 + hO];
-      if (!(ok = warp_wait<true>(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
+      if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
       tc_fence_after();
       const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
       const size_t row0 = (size_t)(sg.b * p.s_q + qrow) * p.n_h;
       const size_t slot = sg.whole ? 0 : (size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow;
       const int col0 = 256 * c + 128 * (qd >> 1);  // latent column of TMEM column kTmemO + 128c
-      // rows leave through a 2 KB per-warp staging area (the P buffers are
-      // free now) so that each global store instruction writes 64 contiguous
-      // bytes of 8 rows; 16-byte chunks are rotated by (row >> 1) & 3 so that
+      // rows leave through a 1 KB per-warp staging area (the P second-half
+      // ring is free now): each thread stages 32 B of its row, then every global
+      // store instruction writes 32 contiguous bytes of 16 rows; the two
+      // 16-byte halves are swapped on rows with (row >> 2) odd so that
       // neither side of the staging has bank conflicts
-      const uint32_t stg = sbase + kOffP + sw_warp * 2048;
-      const uint32_t my_row = stg + lane * 64;
-      const uint32_t my_rot = static_cast<uint32_t>((lane >> 1) & 3);
-      auto flush = [&](int col_first, bool as_bf16) {
+      const uint32_t stg = sbase + kOffP + sw_warp * 1024;
+      const uint32_t my_row = stg + lane * 32;
+      const uint32_t my_rot = static_cast<uint32_t>((lane >> 2) & 1);
+      auto flush = [&](int col_first) {
         __syncwarp();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int r = (lane >> 2) + 8 * k, ch = lane & 3;
-          const float4 v = ld_shared_v4(stg + r * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
+        for (int k = 0; k < 2; ++k) {
+          const int r = (lane >> 1) + 16 * k, ch = lane & 1;
+          const float4 v = ld_shared_v4(stg + r * 32 + ((ch ^ ((r >> 2) & 1)) << 4));
           const int head = 64 * (int)rank + ((32 * qd + r) & 63);
           if (head < p.n_h) {
-            if (as_bf16)
-              *reinterpret_cast<float4*>(p.u + (row0 + head) * kDc + col_first + 8 * ch) = v;
-            else
-              *reinterpret_cast<float4*>(p.part_u + (slot * p.n_h + head) * kDc + col_first +
-                                         4 * ch) = v;
+            __nv_bfloat16* dst = sg.whole ? p.u + (row0 + head) * kDc
+                                          : p.part_u + (slot * p.n_h + head) * kDc;
+            *reinterpret_cast<float4*>(dst + col_first + 8 * ch) = v;
           }
         }
         __syncwarp();
+      };
+      auto stage = [&](const uint32_t (&w)[8]) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          st_shared_v4(my_row + ((k ^ my_rot) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
+                       w[4 * k + 3]);
       };
       for (int c0 = 0; c0 < 128; c0 += 32) {
         float o[32];
         tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
         tmem_wait_ld();
-        if (sg.whole) {
-          uint32_t w[16];
+        // u of a whole sequence, or this segment's partial u (the combine
+        // stage weights and sums the partials in fp32): bf16 either way
+        for (int hf = 0; hf < 2; ++hf) {  // 16 columns per round
+          uint32_t w[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * e] * inv, o[2 * e + 1] * inv);
+          for (int e = 0; e < 8; ++e) {
+            const __nv_bfloat162 h2 =
+                __floats2bfloat162_rn(o[16 * hf + 2 * e] * inv, o[16 * hf + 2 * e + 1] * inv);
             w[e] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            st_shared_v4(my_row + ((k ^ my_rot) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
-                         w[4 * k + 3]);
-          flush(col0 + c0, true);
-        } else {
-          for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float* v = o + 16 * hf + 4 * k;
-              st_shared_v4(my_row + ((k ^ my_rot) << 4), __float_as_uint(v[0] * inv),
-                           __float_as_uint(v[1] * inv), __float_as_uint(v[2] * inv),
-                           __float_as_uint(v[3] * inv));
-            }
-            flush(col0 + c0 + 16 * hf, false);
-          }
+          stage(w);
+          flush(col0 + c0 + 16 * hf);
         }
       }
       const int head = 64 * (int)rank + hO;
@@ -706,7 +758,7 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   p.header = a.header;
   p.tile_prefix = a.tile_prefix;
   p.split_base = a.split_base;
-  p.part_u = a.part_u;
+  p.part_u = reinterpret_cast<__nv_bfloat16*>(a.part_u);
   p.part_lse = a.part_lse;
   p.u = static_cast<__nv_bfloat16*>(a.u);
   p.lse = a.lse;

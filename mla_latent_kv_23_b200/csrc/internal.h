@@ -39,6 +39,7 @@ struct DecodeArgs {
   int B, s_q, n_h, d_c, d_R, page_size, max_pages, num_pages, num_chunks;
   float scale;
   bool bf16;
+  bool part_bf16;  // split partials of u are stored as bf16 (tensor-core path) instead of fp32
 };
 
 cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s);

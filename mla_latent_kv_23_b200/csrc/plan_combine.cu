@@ -108,13 +108,26 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Four consecutive partial values as floats (partials are fp32, or bf16 when
+// the attend stage stored them so).
+template <bool kPartBf16>
+__device__ __forceinline__ float4 load4(const void* base, size_t idx) {
+  if (kPartBf16) {
+    const uint2 r = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + idx);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
+  return *reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+}
+
 // One warp per output row (b, r, head).  Lane s holds the weight of split s
 // (32 at a time); the column loop broadcasts it with a shuffle, so every
-// split costs one exp per row and one float4 load per lane per 128 columns.
-template <bool kBf16>
+// split costs one exp per row and one 4-value load per lane per 128 columns.
+template <bool kBf16, bool kPartBf16>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const int* __restrict__ tile_prefix, const int* __restrict__ split_base,
-                   const float* __restrict__ part_u, const float* __restrict__ part_lse,
+                   const void* __restrict__ part_u, const float* __restrict__ part_lse,
                    void* __restrict__ u_out, float* __restrict__ lse_out, int s_q, int n_h,
                    int d_c, int rows) {
   ptx::pdl_wait_previous();
@@ -148,7 +161,7 @@ __global__ void __launch_bounds__(kCombineThreads)
         for (int k = 0; k < n_here; ++k) {
           const float w = __shfl_sync(0xffffffffu, w_me, k);
           const size_t slot = slot0 + (size_t)(s0 + k) * s_q;
-          const float4 v = *reinterpret_cast<const float4*>(part_u + (slot * n_h + h) * d_c + c);
+          const float4 v = load4<kPartBf16>(part_u, (slot * n_h + h) * d_c + c);
           acc.x += w * v.x;
           acc.y += w * v.y;
           acc.z += w * v.z;
@@ -191,13 +204,18 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const int* tp = a.tile_prefix;
+  const int* sb = a.split_base;
+  const void* pu = a.part_u;
+  const float* pl = a.part_lse;
+  if (a.bf16 && a.part_bf16)
+    return cudaLaunchKernelEx(&cfg, combine_kernel<true, true>, tp, sb, pu, pl, a.u, a.lse, a.s_q,
+                              a.n_h, a.d_c, rows);
   if (a.bf16)
-    return cudaLaunchKernelEx(&cfg, combine_kernel<true>, (const int*)a.tile_prefix,
-                              (const int*)a.split_base, (const float*)a.part_u,
-                              (const float*)a.part_lse, a.u, a.lse, a.s_q, a.n_h, a.d_c, rows);
-  return cudaLaunchKernelEx(&cfg, combine_kernel<false>, (const int*)a.tile_prefix,
-                            (const int*)a.split_base, (const float*)a.part_u,
-                            (const float*)a.part_lse, a.u, a.lse, a.s_q, a.n_h, a.d_c, rows);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<true, false>, tp, sb, pu, pl, a.u, a.lse, a.s_q,
+                              a.n_h, a.d_c, rows);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<false, false>, tp, sb, pu, pl, a.u, a.lse, a.s_q,
+                            a.n_h, a.d_c, rows);
 }
 
 }  // namespace mla

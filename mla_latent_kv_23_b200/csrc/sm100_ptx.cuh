@@ -10,12 +10,16 @@
 namespace mla {
 namespace ptx {
 
-// Longest any single wait may take before the kernel gives up (ns).
-constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+// Longest any single wait may take before the kernel gives up, in SM clock
+// cycles (about one second at the B200 boost clock, two at 1 GHz).  Cycles
+// are counted with clock64, which is cheap to read; the global timer is not.
+constexpr uint64_t kWaitLimitCycles = 2000ull * 1000ull * 1000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+__device__ __forceinline__ uint64_t cycles() { return static_cast<uint64_t>(clock64()); }
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -94,16 +98,19 @@ __device__ __forceinline__ bool mbar_test_nb_cluster(uint32_t bar, uint32_t pari
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and ORs `flag` into *err) if that takes longer than kWaitLimitNs.
+// (and ORs `flag` into *err) if that takes longer than kWaitLimitCycles.
+// Polls with the non-blocking test_wait: the potentially-suspending try_wait
+// was measured to add hundreds of ns of wake-up latency to hand-offs between
+// warps of this kernel, even for phases that had already completed.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int flag) {
-  if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  if (kCluster ? mbar_test_nb_cluster(bar, parity) : mbar_test_nb(bar, parity)) return true;
+  const uint64_t t0 = cycles();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+      if (kCluster ? mbar_test_nb_cluster(bar, parity) : mbar_test_nb(bar, parity)) return true;
+    if (cycles() - t0 > kWaitLimitCycles) {
       atomicOr(err, flag);
       return false;
     }
@@ -122,6 +129,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+// 2D tiled load into this CTA's shared memory whose byte count completes on
+// a barrier of the even CTA of the pair (`cluster_bar`, a shared::cluster
+// address): the operand half a paired MMA reads from this CTA.  No multicast.
+__device__ __forceinline__ void tma_load_2d_to_pair(uint32_t dst, const CUtensorMap* m,
+                                                    uint32_t cluster_bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(cluster_bar), "r"(x), "r"(y)
       : "memory");
 }
 // 3D tiled load (x inner, then y, then z).
@@ -170,6 +188,16 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, floa
           cluster_addr),
       "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
       : "memory");
+}
+// Asynchronous 4-byte store into shared memory of a CTA in the cluster whose
+// completion is counted (4 bytes) on that CTA's mbarrier; the count carries
+// release semantics at cluster scope, and the issuing thread does not wait.
+// Used as a non-blocking cross-CTA arrival (the stored word is not read).
+__device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   cluster_addr),
+               "r"(v), "r"(cluster_bar)
+               : "memory");
 }
 __device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
   float4 v;

@@ -120,6 +120,12 @@ def check_expanded(w, inp, out, picks=None):
 # (a weight error moves a whole cached row, so it reaches o through W^UV).
 # The checks allow 2x these.
 def tight_u_bound(u_ref, abs_c):
+    """Rounding budget of the bf16 path for u_i = sum_j a_j c_j, with
+    abs_c = sum_j a_j |c_j|: the bf16 weights P (relative 2^-9 each, so at most
+    2^-9 abs_c), the bf16 split partials the combine stage merges (each within
+    2^-9 of itself, and the split weights sum to 1, so at most 2^-9 abs_c
+    again) and the final bf16 u (2^-9 |u|); doubled for fp32 accumulation
+    order."""
     return 2.0 * (2.0 ** -8 * abs_c + 2.0 ** -9 * np.abs(u_ref)) + 1e-6
 
 
