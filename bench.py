@@ -104,7 +104,7 @@ class ClockSampler:
                "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period_s: float = 0.002):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.samples = []
         self.period = period_s
         self.ok = False
@@ -146,9 +146,9 @@ class ClockSampler:
         t0, t1 = self._mark
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
         window = "timed region"
-        if len(inside) < 3:   # a short timed region: widen to the busy window around it
-            inside = [s for s in self.samples if t0 - 0.5 <= s[0] <= t1]
-            window = "timed region + 0.5 s of warm-up before it"
+        if len(inside) < 3:   # a short timed region: add the soak replays right before it
+            inside = [s for s in self.samples if t0 - 0.1 <= s[0] <= t1]
+            window = "timed region + up to 0.1 s of identical untimed replays just before it"
         busy = [s for s in inside if not (s[2] & self.REASONS["gpu_idle"])] or inside
         reasons = sorted({n for s in busy for n, bit in self.REASONS.items()
                           if s[2] & bit and n != "gpu_idle"})
@@ -310,6 +310,16 @@ def run_gpu(args, w):
         for k in range(args.warmup):
             graphs[k % R].replay()
     stream.synchronize()
+    # untimed soak of the same replays (~50 ms) so that the clock sampler has
+    # readings of the loaded GPU right up to the timed region
+    soak_until = time.perf_counter() + 0.05
+    with torch.cuda.stream(stream):
+        k = 0
+        while time.perf_counter() < soak_until:
+            for _ in range(16):
+                graphs[k % R].replay()
+                k += 1
+            stream.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)

@@ -15,7 +15,7 @@
 namespace mla {
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;
 
 // Inclusive scan of one int per thread across the block; returns the
 // thread's inclusive value and writes the block total to *total.
@@ -184,6 +184,95 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (lse_out != nullptr && lane == 0) lse_out[static_cast<size_t>(br) * n_h + h] = lse_all;
 }
 
+// Merge of bf16 partials with d_c = 512 (the tensor-core path).  One warp per
+// output row; lane l owns columns [16 l, 16 l + 16).  The partials of up to 8
+// splits are loaded before any is used, so a row waits for memory about once
+// per 8 splits instead of once per split.
+template <bool kBf16>
+__global__ void __launch_bounds__(kCombineThreads)
+    combine512_kernel(const int* __restrict__ tile_prefix, const int* __restrict__ split_base,
+                      const __nv_bfloat16* __restrict__ part_u, const float* __restrict__ part_lse,
+                      void* __restrict__ u_out, float* __restrict__ lse_out, int s_q, int n_h,
+                      int rows) {
+  constexpr int kDc = 512;
+  ptx::pdl_wait_previous();
+  ptx::pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int h = row % n_h, br = row / n_h;
+  const int b = br / s_q, r = br % s_q;
+  const int nsplit = split_base[b + 1] - split_base[b];
+  const bool empty = tile_prefix[b + 1] == tile_prefix[b];
+  if (nsplit == 0 && !empty) return;  // written directly by the attend stage
+  const size_t slot0 = static_cast<size_t>(split_base[b]) * s_q + r;  // slot of split s: slot0 + s*s_q
+  auto lse_of = [&](int s) { return part_lse[(slot0 + (size_t)s * s_q) * n_h + h]; };
+  // one pass: per-lane running (max, sum of exp), then the warp's
+  float m = -INFINITY, z = 0.f;
+  for (int s = lane; s < nsplit; s += 32) {
+    const float x = lse_of(s);
+    if (x > m) {
+      z = z * expf(m - x) + 1.f;
+      m = x;
+    } else if (x != -INFINITY) {
+      z += expf(x - m);
+    }
+  }
+  const float m_all = warp_max(m);
+  z = warp_sum(m == -INFINITY ? 0.f : z * expf(m - m_all));
+  const float lse_all = (m_all == -INFINITY) ? -INFINITY : m_all + logf(z);
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  if (m_all != -INFINITY) {
+    for (int s0 = 0; s0 < nsplit; s0 += 8) {
+      const int n_here = min(8, nsplit - s0);
+      const float w_me = lane < n_here ? expf(lse_of(s0 + lane) - lse_all) : 0.f;
+      uint4 v[8][2];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < n_here) {
+          const __nv_bfloat16* src =
+              part_u + ((slot0 + (size_t)(s0 + k) * s_q) * n_h + h) * kDc + 16 * lane;
+          v[k][0] = *reinterpret_cast<const uint4*>(src);
+          v[k][1] = *reinterpret_cast<const uint4*>(src + 8);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float w = __shfl_sync(0xffffffffu, w_me, k);
+        if (k < n_here) {
+          const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(v[k]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 f = __bfloat1622float2(x[e]);
+            acc[2 * e] += w * f.x;
+            acc[2 * e + 1] += w * f.y;
+          }
+        }
+      }
+    }
+  }
+  const size_t orow = static_cast<size_t>(br) * n_h + h;
+  if (kBf16) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const __nv_bfloat162 t = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+      pk[e] = *reinterpret_cast<const uint32_t*>(&t);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(u_out) + orow * kDc + 16 * lane);
+    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  } else {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(u_out) + orow * kDc + 16 * lane);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+  }
+  if (lse_out != nullptr && lane == 0) lse_out[orow] = lse_all;
+}
+
 }  // namespace
 
 cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s) {
@@ -208,6 +297,14 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
   const int* sb = a.split_base;
   const void* pu = a.part_u;
   const float* pl = a.part_lse;
+  if (a.part_bf16 && a.d_c == 512) {
+    const __nv_bfloat16* pb = static_cast<const __nv_bfloat16*>(pu);
+    if (a.bf16)
+      return cudaLaunchKernelEx(&cfg, combine512_kernel<true>, tp, sb, pb, pl, a.u, a.lse, a.s_q,
+                                a.n_h, rows);
+    return cudaLaunchKernelEx(&cfg, combine512_kernel<false>, tp, sb, pb, pl, a.u, a.lse, a.s_q,
+                              a.n_h, rows);
+  }
   if (a.bf16 && a.part_bf16)
     return cudaLaunchKernelEx(&cfg, combine_kernel<true, true>, tp, sb, pu, pl, a.u, a.lse, a.s_q,
                               a.n_h, a.d_c, rows);
