@@ -131,6 +131,7 @@ __device__ __forceinline__ int lat_col(int kc, int half) {
 
 struct Params {
   Sm100Maps maps;
+  const __nv_bfloat16* q;  // [B * s_q, n_h, 576], for L2 prefetch of the next segment's rows
   const int* block_table;
   const int* seqlens;
   const int* header;
@@ -344,6 +345,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
       }
       q_in_flight = true;
+      // the next segment's query rows go to L2 now, so that its TMA load
+      // after this segment's last S is an L2 hit
+      if (lane == 0) {
+        ChunkWalk peek = walk;
+        Segment nx;
+        const int heads = min(64, p.n_h - 64 * (int)rank);
+        if (heads > 0 && peek.next(nx)) {
+          const __nv_bfloat16* src =
+              p.q + ((size_t)(nx.b * p.s_q + qrow) * p.n_h + 64 * rank) * (kDc + 64);
+          const uint32_t bytes = static_cast<uint32_t>(heads) * (kDc + 64) * 2;
+          for (uint32_t off = 0; off < bytes; off += 16384)
+            bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(src) + off, min(16384u, bytes - off));
+        }
+      }
       if (!(ok = warp_wait(bar(Q_LOCAL), seg_i & 1, p.err))) break;
       q_in_flight = false;
       if (lane == 0) signal_lead(Q_FULL, true, 4u, 8);
@@ -753,6 +768,7 @@ int decode_sm100_prepare() {
 cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s) {
   Params p;
   p.maps = maps;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.block_table = a.block_table;
   p.seqlens = a.seqlens;
   p.header = a.header;

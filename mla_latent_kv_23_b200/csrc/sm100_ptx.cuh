@@ -152,6 +152,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// Asks the L2 to fetch `bytes` (multiple of 16, 16-byte aligned) of global
+// memory ahead of use; nothing is written anywhere else.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
+
 // Generic-proxy writes to shared memory become visible to the async proxy
 // (tensor core / TMA) after this fence.
 __device__ __forceinline__ void fence_proxy_async_smem() {
