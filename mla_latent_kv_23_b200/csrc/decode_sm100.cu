@@ -117,7 +117,7 @@ constexpr size_t kSmemBytes = kSmemUsed;  // the base is 1024-byte aligned (chec
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;     // 2 x 128 columns
 constexpr uint32_t kTmemO = 256;   // 2 x 128 columns (latent blocks 0-255, 256-511)
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
+constexpr float kRescaleThreshold = 30.0f;  // log2 units: rescale O only if the max grows by > 2^30
 constexpr uint16_t kBothCtas = 3;
 
 static_assert(kOffKv % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "align");

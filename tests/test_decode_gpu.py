@@ -112,6 +112,32 @@ def test_decode_on_exact_inputs_tight(s_q, splits):
     assert_tight(check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"]))
 
 
+@pytest.mark.parametrize("s_q,splits", [(1, 0), (1, 4), (2, 0)])
+def test_running_max_jumps_across_tiles(s_q, splits):
+    # The kernel keeps a stale running maximum and rescales O and the row sum
+    # only when a tile's maximum exceeds it by a large factor.  Make every
+    # head's score climb tile by tile: steps of about 2^20 (below that factor:
+    # weights up to 2^20 accumulate unrescaled), 2^40 and 2^50 (above it: the
+    # rescale must run), and drops (the maximum stays).  A skipped or wrong
+    # rescale leaves earlier tiles weighted 2^30+ times too high.
+    w = v3_small(s_q=s_q, B=3, seqlens=(1000, 777, 130))
+    inp = synth.draw(w)
+    q = synth.random_q(w)
+    q[..., 0] = 16.0
+    cache = inp["cache"].copy()
+    rng = np.random.default_rng(5)
+    for b, L in enumerate(inp["seqlens"]):
+        n_t = (int(L) + 63) // 64
+        gamma = np.cumsum(rng.choice([-12.0, 12.0, 24.0, 30.0], size=n_t))
+        gamma -= gamma.min()
+        rows = synth.cache_row_ids(w, inp["block_table"], b, int(L))
+        cache[rows, 0] = gamma[np.arange(int(L)) // 64]
+    inp["cache"] = synth.bf16_round(cache)
+    out = run_pipeline(w, inp, num_splits=splits, q=to_dev(q, w))
+    picks = [(b, r, i) for b in range(w.B) for r in range(s_q) for i in (0, 1, 64, 127)]
+    assert_tight(check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"]))
+
+
 @pytest.mark.parametrize("T", [1, 16, 64, 100])
 def test_up_projection_on_exact_input(T):
     # the up-projection judged on its own bf16 input u (from the generator)
