@@ -127,6 +127,7 @@ int choose_chunks(const mla_decode_params* p, const DeviceInfo* d) {
 
 struct Resolved {
   DecodeArgs a;
+  long long slots = 0;  // partial rows per head the workspace holds
   bool tc = false;
   const DeviceInfo* dev = nullptr;
 };
@@ -141,6 +142,7 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MLA_ERR_INVALID_ARG;
   uint8_t* w = static_cast<uint8_t*>(ws);
+  r->slots = L.slots;
   DecodeArgs& a = r->a;
   a.q = p->q;
   a.kv = p->kv_cache;
@@ -151,6 +153,8 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   a.header = reinterpret_cast<int*>(w + L.header);
   a.tile_prefix = reinterpret_cast<int*>(w + L.tile_prefix);
   a.split_base = reinterpret_cast<int*>(w + L.split_base);
+  a.chunk_t = reinterpret_cast<int*>(w + L.chunk_t);
+  a.chunk_b = reinterpret_cast<int*>(w + L.chunk_b);
   a.part_lse = reinterpret_cast<float*>(w + L.part_lse);
   a.part_u = reinterpret_cast<float*>(w + L.part_u);
   a.err = r->dev->flags;
@@ -195,6 +199,19 @@ mla_status encode_q(CUtensorMap* m, const void* ptr, uint64_t n_h, uint64_t qrow
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// 3D map over an output [rows, n_h, 512] (bf16) for TMA stores: box 64 x 32
+// heads x 1, 128-byte swizzle.
+mla_status encode_out(CUtensorMap* m, void* ptr, uint64_t n_h, uint64_t rows) {
+  const cuuint64_t dims[3] = {512, n_h, rows};
+  const cuuint64_t strides[2] = {512 * 2, n_h * 512 * 2};
+  const cuuint32_t box[3] = {64, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s) {
   if (!r.tc) return cuda_status(launch_decode_simt(r.a, s));
   Sm100Maps maps;
@@ -206,6 +223,9 @@ mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s)
   const uint64_t qrows = (uint64_t)p->B * p->s_q;
   if ((st = encode_q(&maps.q_lat, p->q, p->n_h, qrows, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
       (st = encode_q(&maps.q_rope, p->q, p->n_h, qrows, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+    return st;
+  if ((st = encode_out(&maps.u_out, p->u, p->n_h, qrows)) != MLA_OK ||
+      (st = encode_out(&maps.part_out, r.a.part_u, p->n_h, (uint64_t)r.slots)) != MLA_OK)
     return st;
   return cuda_status(launch_decode_sm100(r.a, maps, s));
 }
@@ -222,6 +242,10 @@ WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks) {
   off = align_up(off + sizeof(int) * (B + 1), 256);
   L.split_base = off;
   off = align_up(off + sizeof(int) * (B + 1), 256);
+  L.chunk_t = off;
+  off = align_up(off + sizeof(int) * (num_chunks + 1), 256);
+  L.chunk_b = off;
+  off = align_up(off + sizeof(int) * num_chunks, 256);
   L.part_lse = off;
   off = align_up(off + sizeof(float) * (size_t)L.slots * n_h, 256);
   L.part_u = off;

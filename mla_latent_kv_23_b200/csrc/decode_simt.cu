@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
   const T* kv = static_cast<const T*>(a.kv);
 
   ChunkWalk walk;
-  walk.init(a.tile_prefix, a.B, chunk, a.header[1]);
+  walk.init(a.tile_prefix, a.chunk_t, a.chunk_b, a.header, a.B, chunk);
   Segment sg;
   while (walk.next(sg)) {
     const int b = sg.b;

@@ -56,8 +56,13 @@
 // tile.  O rows are rescaled by the warp that can reach their TMEM lanes,
 // which derives the same maximum from the same shared values.
 //
-// Work: the plan stage cuts the batch's tiles into equal chunks; cluster c
-// handles chunk c / s_q for query row c % s_q, walking its segments in order.
+// Epilogue: u = O / l leaves TMEM through the query area (free once the
+// segment's last S is done) by TMA stores of whole 128-byte lines; the relay
+// loads the next segment's query after those stores have read it.
+//
+// Work: the plan stage cuts the batch's tiles into chunks of equal cost
+// (tiles plus a fixed charge per sequence start); cluster c handles chunk
+// c / s_q for query row c % s_q, walking its segments in order.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -106,6 +111,7 @@ enum Bar {
   Q_FULL,                          // even CTA, paired: both queries in place (relays)
   Q_EMPTY,                         // last S of a segment done (paired commit)
   GRP,                             // the 8 softmax warps of this CTA
+  EPI_FREE,                        // the 8 softmax warps' output stores have read the query area
   MMA_FINAL,                       // even CTA: all S issued so far are complete
   MMA_FINAL_PV,                    // even CTA: all P . C issued so far are complete
   BAR_COUNT
@@ -137,9 +143,9 @@ struct Params {
   const int* header;
   const int* tile_prefix;
   const int* split_base;
-  __nv_bfloat16* part_u;  // split partials of u, bf16
+  const int* chunk_t;
+  const int* chunk_b;
   float* part_lse;
-  __nv_bfloat16* u;
   float* lse;
   int* err;
   int B, s_q, n_h, max_pages, page_size, num_pages;
@@ -220,6 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(Q_EMPTY), 1);
     mbar_init(bar(GRP), 8);
+    mbar_init(bar(EPI_FREE), 8);
     mbar_init(bar(MMA_FINAL), 1);
     mbar_init(bar(MMA_FINAL_PV), 1);
     fence_mbar_init();
@@ -244,12 +251,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // everything above overlaps the plan kernel; its results are read below
   pdl_wait_previous();
   pdl_launch_dependents();
-  const int cs = p.header[1];
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ producer
     ChunkWalk walk;
-    walk.init(p.tile_prefix, p.B, chunk, cs);
+    walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
     Segment sg;
     int g = 0;
     int last_n[kStages], tail_n[kStages];  // uses of LOCAL_FULL per stage
@@ -318,7 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpRelay) {
     // ------------------------------------------------------------ relay
     ChunkWalk walk;
-    walk.init(p.tile_prefix, p.B, chunk, cs);
+    walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
     Segment sg;
     int g = 0, seg_i = 0;
     int tail_n[kStages];  // uses of LOCAL_FULL per stage, in tile order
@@ -329,7 +335,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // this segment's query rows (h, j) = Q[64 rank + 16 qd + i, columns of
       // CTA j], stored as row 32 qd + 16 j + i; heads >= n_h read as zero
       // (the tensor map ends there)
-      if (seg_i > 0 && !(ok = warp_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err))) break;
+      // the query area is free once the previous segment's last S has read
+      // it and its epilogue's output stores (staged there) have left
+      if (seg_i > 0 && !(ok = warp_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err) &&
+                              warp_wait(bar(EPI_FREE), (seg_i - 1) & 1, p.err)))
+        break;
       if (lane == 0) {
         const int z = sg.b * p.s_q + qrow;
         mbar_arrive_expect_tx(bar(Q_LOCAL), kQBytes);
@@ -403,7 +413,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdS = idesc_bf16(256, 128, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, 256, true);
       ChunkWalk walk;
-      walk.init(p.tile_prefix, p.B, chunk, cs);
+      walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
       Segment sg;
       int g0 = 0, seg_i = 0;
       bool ok = true;
@@ -511,7 +521,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
 
     ChunkWalk walk;
-    walk.init(p.tile_prefix, p.B, chunk, cs);
+    walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
     Segment sg;
     int g = 0;
     bool ok = true;
@@ -519,6 +529,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int L = p.seqlens[sg.b];
       const int L_eff = L - p.s_q + 1 + qrow;  // positions this query row may see
       const int n_t = sg.t1 - sg.t0;
+      // the segment's output row: u's row, or its partial slot (read now,
+      // used by the epilogue)
+      const int out_z =
+          sg.whole ? sg.b * p.s_q + qrow : (p.split_base[sg.b] + sg.part) * p.s_q + qrow;
       // m_s: running max of the S head (weights); m_o: the same sequence of
       // values for the O head (rescaling), derived from the same shared maxima
       float m_s = -INFINITY, m_o = -INFINITY, l = 0.f, l_exact = 0.f;
@@ -657,67 +671,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
       tc_fence_after();
       const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
-      const size_t row0 = (size_t)(sg.b * p.s_q + qrow) * p.n_h;
-      const size_t slot = sg.whole ? 0 : (size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow;
       const int col0 = 256 * c + 128 * (qd >> 1);  // latent column of TMEM column kTmemO + 128c
-      // rows leave through a 1 KB per-warp staging area (the P second-half
-      // ring is free now): each thread stages 32 B of its row, then every global
-      // store instruction writes 32 contiguous bytes of 16 rows; the two
-      // 16-byte halves are swapped on rows with (row >> 2) odd so that
-      // neither side of the staging has bank conflicts
-      const uint32_t stg = sbase + kOffP + sw_warp * 1024;
-      const uint32_t my_row = stg + lane * 32;
-      const uint32_t my_rot = static_cast<uint32_t>((lane >> 2) & 1);
-      auto flush = [&](int col_first) {
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int r = (lane >> 1) + 16 * k, ch = lane & 1;
-          const float4 v = ld_shared_v4(stg + r * 32 + ((ch ^ ((r >> 2) & 1)) << 4));
-          const int head = 64 * (int)rank + ((32 * qd + r) & 63);
-          if (head < p.n_h) {
-            __nv_bfloat16* dst = sg.whole ? p.u + (row0 + head) * kDc
-                                          : p.part_u + (slot * p.n_h + head) * kDc;
-            *reinterpret_cast<float4*>(dst + col_first + 8 * ch) = v;
-          }
-        }
-        __syncwarp();
-      };
-      auto stage = [&](const uint32_t (&w)[8]) {
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-          st_shared_v4(my_row + ((k ^ my_rot) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
-                       w[4 * k + 3]);
-      };
+      // The segment's last S has read Q, so the query area stages the output:
+      // 8 KB per warp, its 32 heads x 128 columns as two boxes of 64 columns
+      // in the 128-byte-swizzled layout of the output tensor map (row = head =
+      // lane, 16-byte chunk k of a row at k ^ (row & 7)).  Each box leaves by
+      // one TMA store, which writes whole 128-byte lines of u; the relay loads
+      // the next segment's query only after the stores have read the area.
+      const uint32_t stg = sbase + kOffQ + sw_warp * 8192u;
+      const int y_head = 64 * (int)rank + 32 * (qd & 1);  // first head of this warp's rows
+      const CUtensorMap* omap = sg.whole ? &p.maps.u_out : &p.maps.part_out;
       for (int c0 = 0; c0 < 128; c0 += 32) {
         float o[32];
         tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
         tmem_wait_ld();
         // u of a whole sequence, or this segment's partial u (the combine
         // stage weights and sums the partials in fp32): bf16 either way
-        for (int hf = 0; hf < 2; ++hf) {  // 16 columns per round
-          uint32_t w[8];
+        const uint32_t row = stg + static_cast<uint32_t>(c0 >> 6) * 4096u + lane * 128u;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
             const __nv_bfloat162 h2 =
-                __floats2bfloat162_rn(o[16 * hf + 2 * e] * inv, o[16 * hf + 2 * e + 1] * inv);
-            w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                __floats2bfloat162_rn(o[8 * e + 2 * k] * inv, o[8 * e + 2 * k + 1] * inv);
+            w[k] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          stage(w);
-          flush(col0 + c0 + 16 * hf);
+          const uint32_t chunk16 = static_cast<uint32_t>(((c0 & 63) >> 3) + e);
+          st_shared_v4(row + ((chunk16 ^ static_cast<uint32_t>(lane & 7)) << 4), w[0], w[1], w[2],
+                       w[3]);
+        }
+        if (c0 & 32) {  // box c0 >> 6 is complete
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && y_head < p.n_h) {
+            tma_store_3d(omap, stg + static_cast<uint32_t>(c0 >> 6) * 4096u, col0 + (c0 & 64),
+                         y_head, out_z);
+            bulk_commit();
+          }
         }
       }
       const int head = 64 * (int)rank + hO;
       if (head < p.n_h && qd < 2 && c == 0) {
         const float lse = le_o > 0.f ? (m_o + log2f(le_o)) * 0.69314718055994531f : -INFINITY;
         if (sg.whole) {
-          if (p.lse != nullptr) p.lse[row0 + head] = lse;
+          if (p.lse != nullptr) p.lse[(size_t)out_z * p.n_h + head] = lse;
         } else {
-          p.part_lse[slot * p.n_h + head] = lse;
+          p.part_lse[(size_t)out_z * p.n_h + head] = lse;
         }
       }
+      // the query area may take the next segment's rows once the stores have
+      // read it
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(EPI_FREE));
       tc_fence_before();
     }
+    // the last stores complete before the CTA exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
@@ -774,9 +786,9 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   p.header = a.header;
   p.tile_prefix = a.tile_prefix;
   p.split_base = a.split_base;
-  p.part_u = reinterpret_cast<__nv_bfloat16*>(a.part_u);
+  p.chunk_t = a.chunk_t;
+  p.chunk_b = a.chunk_b;
   p.part_lse = a.part_lse;
-  p.u = static_cast<__nv_bfloat16*>(a.u);
   p.lse = a.lse;
   p.err = a.err;
   p.B = a.B;

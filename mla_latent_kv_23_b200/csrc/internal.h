@@ -14,10 +14,19 @@ namespace mla {
 constexpr int kTileTokens = 64;   // cache rows per attention tile
 constexpr int kMaxHeads = 128;    // query heads packed as the MMA M dimension
 
-// Workspace of mla_decode.  Header ints: [0] total tiles, [1] tiles per chunk,
-// [2] number of chunks, [3] split rows in use.
+// Cost of starting one more sequence inside a KV chunk (loading its queries,
+// writing its output), in units of one 64-token tile.  The plan cuts chunks on
+// a line where every sequence start takes this many units on top of its tiles,
+// so chunks that hold several sequences get fewer tiles.
+constexpr int kSegCostTiles = 4;
+
+// Workspace of mla_decode.  Header ints: [0] total tiles, [1] line units per
+// chunk, [2] number of chunks, [3] split rows in use, [4] units per sequence
+// start.  chunk_t[c] is the first tile of chunk c (chunk_t[chunks] = total
+// tiles), chunk_b[c] the sequence that tile belongs to.
 struct WsLayout {
-  size_t header = 0, tile_prefix = 0, split_base = 0, part_lse = 0, part_u = 0, total = 0;
+  size_t header = 0, tile_prefix = 0, split_base = 0, chunk_t = 0, chunk_b = 0, part_lse = 0,
+         part_u = 0, total = 0;
   long long slots = 0;  // partial (u, lse) rows per head: (B + chunks) * s_q
 };
 WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks);
@@ -33,6 +42,8 @@ struct DecodeArgs {
   int* header;
   int* tile_prefix;
   int* split_base;
+  int* chunk_t;
+  int* chunk_b;
   float* part_u;
   float* part_lse;
   int* err;
@@ -52,8 +63,11 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s);
 // queries [B * s_q, n_h, 576]: latent boxes 64 x 16 heads x 1 (128-byte
 // swizzle), RoPE boxes 32 x 16 heads x 1 (64-byte swizzle); heads past n_h
 // read as zero.
+// out maps over u [B * s_q, n_h, 512] and over the split partials
+// [slots, n_h, 512] (bf16): boxes 64 x 32 heads x 1, 128-byte swizzle, for
+// the TMA stores of the epilogue; heads past n_h are not written.
 struct Sm100Maps {
-  CUtensorMap kv_lat, kv_rope, q_lat, q_rope;
+  CUtensorMap kv_lat, kv_rope, q_lat, q_rope, u_out, part_out;
 };
 cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s);
 size_t decode_sm100_smem_bytes();

@@ -1,7 +1,10 @@
 // Plan and combine stages of mla_decode.
 //
-// plan:    per-sequence tile counts, their prefix sum, the chunk size, and the
-//          first partial row of every sequence that is cut into several
+// plan:    per-sequence tile counts and their prefix sum; the cut of the tile
+//          line into KV chunks (uniform on a line that charges every sequence
+//          start kSegCostTiles units, so a chunk that starts new sequences
+//          takes fewer tiles); the first tile and sequence of every chunk; and
+//          the first partial row of every sequence that is cut into several
 //          chunks (one block; B is small).
 // combine: for every row cut into pieces, merge the partial results by their
 //          log-sum-exp: lse = log sum_s exp(lse_s), u = sum_s exp(lse_s - lse) u_s
@@ -49,10 +52,12 @@ __device__ int block_scan(int v, int* warp_sums, int* total) {
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restrict__ seqlens, int B,
                                                             int s_q, int max_len, int num_chunks,
                                                             int* header, int* tile_prefix,
-                                                            int* split_base, int* err) {
+                                                            int* split_base, int* chunk_t,
+                                                            int* chunk_b, int* err) {
   // let the attend kernel start its prologue while this one runs
   ptx::pdl_launch_dependents();
   __shared__ int warp_sums[32];
+  constexpr int K = kSegCostTiles;
   int carry = 0, total = 0;
   for (int base = 0; base < B; base += blockDim.x) {
     const int i = base + threadIdx.x;
@@ -67,9 +72,30 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
     carry += total;
   }
   const int T = carry;
-  const int cs = T > 0 ? (T + num_chunks - 1) / num_chunks : 1;
+  // the line: sequence b takes units [tp[b] + K b, tp[b + 1] + K (b + 1)),
+  // the first K of them for its start-up; tile t of sequence b is unit
+  // t + K (b + 1)
+  const long long V = (long long)T + (long long)K * B;
+  const int units = V > 0 ? (int)((V + num_chunks - 1) / num_chunks) : 1;
   if (threadIdx.x == 0) tile_prefix[B] = T;
   __syncthreads();
+  // chunk c starts at unit c * units: at the first tile at or after it
+  for (int c = threadIdx.x; c <= num_chunks; c += blockDim.x) {
+    const long long x = (long long)c * units;
+    int t = T, sb = B;
+    if (x < V) {
+      int lo = 0, hi = B;  // largest b with tp[b] + K b <= x
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)tile_prefix[mid] + (long long)K * mid <= x) lo = mid; else hi = mid;
+      }
+      const long long off = x - ((long long)tile_prefix[lo] + (long long)K * (lo + 1));
+      t = tile_prefix[lo] + (off > 0 ? (int)off : 0);
+      sb = lo;
+    }
+    chunk_t[c] = t;
+    if (c < num_chunks) chunk_b[c] = sb;
+  }
   carry = 0;
   for (int base = 0; base < B; base += blockDim.x) {
     const int i = base + threadIdx.x;
@@ -77,7 +103,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
     if (i < B) {
       const int t0 = tile_prefix[i], t1 = tile_prefix[i + 1];
       if (t1 > t0) {
-        const int n = (t1 - 1) / cs - t0 / cs + 1;
+        const long long u0 = (long long)t0 + (long long)K * (i + 1);
+        const int n = (int)((u0 + (t1 - t0) - 1) / units - u0 / units) + 1;
         pieces = n > 1 ? n : 0;
       }
     }
@@ -88,9 +115,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   if (threadIdx.x == 0) {
     split_base[B] = carry;
     header[0] = T;
-    header[1] = cs;
+    header[1] = units;
     header[2] = num_chunks;
     header[3] = carry * s_q;
+    header[4] = K;
   }
 }
 
@@ -195,18 +223,45 @@ __global__ void __launch_bounds__(kCombineThreads)
                       void* __restrict__ u_out, float* __restrict__ lse_out, int s_q, int n_h,
                       int rows) {
   constexpr int kDc = 512;
-  ptx::pdl_wait_previous();
-  ptx::pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  // The plan stage's outputs are read before waiting: that stage completed
+  // before the attend stage that precedes this one passed its own wait, and
+  // this kernel starts only after the attend stage has passed it.
+  int sb0 = 0, sb1 = 0, tp0 = 0, tp1 = 0;
+  int h = 0, br = 0, r = 0;
+  if (row < rows) {
+    h = row % n_h;
+    br = row / n_h;
+    const int b = br / s_q;
+    r = br % s_q;
+    sb0 = split_base[b];
+    sb1 = split_base[b + 1];
+    tp0 = tile_prefix[b];
+    tp1 = tile_prefix[b + 1];
+  }
+  ptx::pdl_wait_previous();
+  ptx::pdl_launch_dependents();
   if (row >= rows) return;
-  const int h = row % n_h, br = row / n_h;
-  const int b = br / s_q, r = br % s_q;
-  const int nsplit = split_base[b + 1] - split_base[b];
-  const bool empty = tile_prefix[b + 1] == tile_prefix[b];
-  if (nsplit == 0 && !empty) return;  // written directly by the attend stage
-  const size_t slot0 = static_cast<size_t>(split_base[b]) * s_q + r;  // slot of split s: slot0 + s*s_q
+  const int nsplit = sb1 - sb0;
+  if (nsplit == 0 && tp1 != tp0) return;  // written directly by the attend stage
+  const size_t slot0 = static_cast<size_t>(sb0) * s_q + r;  // slot of split s: slot0 + s*s_q
   auto lse_of = [&](int s) { return part_lse[(slot0 + (size_t)s * s_q) * n_h + h]; };
+  auto load_group = [&](int s0, uint4 (&v)[8][2]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (s0 + k < nsplit) {
+        const __nv_bfloat16* src =
+            part_u + ((slot0 + (size_t)(s0 + k) * s_q) * n_h + h) * kDc + 16 * lane;
+        v[k][0] = *reinterpret_cast<const uint4*>(src);
+        v[k][1] = *reinterpret_cast<const uint4*>(src + 8);
+      }
+    }
+  };
+  // the first 8 partial rows are requested together with the statistics, so
+  // one memory round trip covers rows with up to 8 pieces
+  uint4 v[8][2];
+  load_group(0, v);
   // one pass: per-lane running (max, sum of exp), then the warp's
   float m = -INFINITY, z = 0.f;
   for (int s = lane; s < nsplit; s += 32) {
@@ -226,18 +281,9 @@ __global__ void __launch_bounds__(kCombineThreads)
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   if (m_all != -INFINITY) {
     for (int s0 = 0; s0 < nsplit; s0 += 8) {
+      if (s0 > 0) load_group(s0, v);
       const int n_here = min(8, nsplit - s0);
       const float w_me = lane < n_here ? expf(lse_of(s0 + lane) - lse_all) : 0.f;
-      uint4 v[8][2];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (k < n_here) {
-          const __nv_bfloat16* src =
-              part_u + ((slot0 + (size_t)(s0 + k) * s_q) * n_h + h) * kDc + 16 * lane;
-          v[k][0] = *reinterpret_cast<const uint4*>(src);
-          v[k][1] = *reinterpret_cast<const uint4*>(src + 8);
-        }
-      }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float w = __shfl_sync(0xffffffffu, w_me, k);
@@ -278,7 +324,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s) {
   plan_kernel<<<1, kPlanThreads, 0, s>>>(a.seqlens, a.B, a.s_q, a.max_pages * a.page_size,
                                          a.num_chunks, a.header, a.tile_prefix, a.split_base,
-                                         a.err);
+                                         a.chunk_t, a.chunk_b, a.err);
   return cudaGetLastError();
 }
 
