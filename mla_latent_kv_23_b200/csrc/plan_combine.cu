@@ -19,6 +19,7 @@ namespace mla {
 namespace {
 
 constexpr int kPlanThreads = 256;
+constexpr int kPlanSmemSeqs = 4096;  // batches up to this size keep the tile prefix on chip
 
 // Inclusive scan of one int per thread across the block; returns the
 // thread's inclusive value and writes the block total to *total.
@@ -57,6 +58,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   // let the attend kernel start its prologue while this one runs
   ptx::pdl_launch_dependents();
   __shared__ int warp_sums[32];
+  __shared__ int tp_s[kPlanSmemSeqs + 1];
+  const bool on_chip = B <= kPlanSmemSeqs;
   constexpr int K = kSegCostTiles;
   int carry = 0, total = 0;
   for (int base = 0; base < B; base += blockDim.x) {
@@ -68,7 +71,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
       else tiles = (L + kTileTokens - 1) / kTileTokens;
     }
     const int incl = block_scan(tiles, warp_sums, &total);
-    if (i < B) tile_prefix[i] = carry + incl - tiles;
+    if (i < B) {
+      tile_prefix[i] = carry + incl - tiles;
+      if (on_chip) tp_s[i] = carry + incl - tiles;
+    }
     carry += total;
   }
   const int T = carry;
@@ -77,8 +83,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   // t + K (b + 1)
   const long long V = (long long)T + (long long)K * B;
   const int units = V > 0 ? (int)((V + num_chunks - 1) / num_chunks) : 1;
-  if (threadIdx.x == 0) tile_prefix[B] = T;
+  if (threadIdx.x == 0) {
+    tile_prefix[B] = T;
+    if (on_chip) tp_s[B] = T;
+  }
   __syncthreads();
+  // the searches below read the prefix from shared memory when it fits
+  const int* tp = on_chip ? tp_s : tile_prefix;
   // chunk c starts at unit c * units: at the first tile at or after it
   for (int c = threadIdx.x; c <= num_chunks; c += blockDim.x) {
     const long long x = (long long)c * units;
@@ -87,10 +98,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
       int lo = 0, hi = B;  // largest b with tp[b] + K b <= x
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if ((long long)tile_prefix[mid] + (long long)K * mid <= x) lo = mid; else hi = mid;
+        if ((long long)tp[mid] + (long long)K * mid <= x) lo = mid; else hi = mid;
       }
-      const long long off = x - ((long long)tile_prefix[lo] + (long long)K * (lo + 1));
-      t = tile_prefix[lo] + (off > 0 ? (int)off : 0);
+      const long long off = x - ((long long)tp[lo] + (long long)K * (lo + 1));
+      t = tp[lo] + (off > 0 ? (int)off : 0);
       sb = lo;
     }
     chunk_t[c] = t;
@@ -101,7 +112,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
     const int i = base + threadIdx.x;
     int pieces = 0;
     if (i < B) {
-      const int t0 = tile_prefix[i], t1 = tile_prefix[i + 1];
+      const int t0 = tp[i], t1 = tp[i + 1];
       if (t1 > t0) {
         const long long u0 = (long long)t0 + (long long)K * (i + 1);
         const int n = (int)((u0 + (t1 - t0) - 1) / units - u0 / units) + 1;
