@@ -267,7 +267,7 @@ def draw(w: Workload, with_weights: bool = True) -> dict:
 def random_q(w: Workload, seed_tag: int = 0) -> np.ndarray:
     """An absorbed query tensor [B, s_q, n_h, d_c + d_R] drawn directly.
 
-    Used where the decode is judged on its own bf16 inputs rather than
+    Used where the decode is checked on its own bf16 inputs rather than
     through query formation: the long-context stress workload and the
     invariance checks.  The latent part is N(0, 0.25) and the RoPE part
     N(0, 1), the spreads the V3-shaped projections of N(0, 1) hidden states

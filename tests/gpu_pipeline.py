@@ -8,7 +8,7 @@ import torch
 from mla_latent_kv_23_b200 import mla, synth
 from oracle import mla_oracle as orc
 
-# spec tolerances: elementwise |gpu - oracle| <= ATOL_REL * (1 + |oracle|);
+# target tolerances: elementwise |gpu - oracle| <= ATOL_REL * (1 + |oracle|);
 # softmax statistics within LSE_REL relative.  "Relative" is taken against
 # max(|lse|, 1): a row with a single cached token has lse = its own score,
 # which can be ~0, where a purely relative test has no meaning.
@@ -157,12 +157,12 @@ def check_absorbed(w, q, inp, out, picks, W_UV=None):
     return res
 
 
-def assert_tight(res, o_north_star=True):
-    """Tight bounds on u (and o when present); the benchmark spec's tolerance on
-    u and lse always, and on o unless o_north_star is False."""
+def assert_tight(res, o_elementwise=True):
+    """Tight bounds on u (and o when present); the elementwise tolerance on
+    u and lse always, and on o unless o_elementwise is False."""
     assert res["u"] <= ATOL_REL, res
     assert res["lse"] <= LSE_REL, res
-    if o_north_star:
+    if o_elementwise:
         assert res["o"] <= ATOL_REL, res
     assert res["tight"] <= 1.0, res
     assert res["tight_o"] <= 1.0, res

@@ -58,7 +58,7 @@ def test_v3_shape_ragged(s_q, splits):
 @pytest.mark.parametrize("s_q,seqlens", [(1, (1, 64, 65, 128, 129)), (2, (2, 64, 65, 130, 3))])
 def test_length_edges(s_q, seqlens):
     # one token, exactly one tile, one tile + 1, two tiles, two tiles + 1;
-    # judged on exact bf16 inputs (q from the generator) with the tight bound
+    # checked on exact bf16 inputs (q from the generator) with the tight bound
     w = v3_small(s_q=s_q, B=len(seqlens), seqlens=seqlens, block_table="identity")
     inp = synth.draw(w)
     q = synth.random_q(w)
@@ -140,7 +140,7 @@ def test_running_max_jumps_across_tiles(s_q, splits):
 
 @pytest.mark.parametrize("T", [1, 16, 64, 100])
 def test_up_projection_on_exact_input(T):
-    # the up-projection judged on its own bf16 input u (from the generator)
+    # the up-projection checked on its own bf16 input u (from the generator)
     w = v3_small(B=T, seqlens=(1,) * T, block_table="identity")
     inp = synth.draw(w)
     u = synth.random_q(w)[:, 0, :, :w.d_c] * 8   # spread up to ~|u| 25 like the stress workload
