@@ -160,7 +160,8 @@ mla_status mla_decode(const mla_decode_params* p, void* workspace, size_t worksp
  * separately; calling them in this order is exactly mla_decode.
  *   plan:    per-sequence tile counts and KV-chunk boundaries into the workspace
  *   attend:  the chunked attention (writes u/lse directly for unsplit rows,
- *            fp32 partials into the workspace otherwise)
+ *            partials into the workspace otherwise: bf16 from the
+ *            tensor-core kernel, fp32 from the CUDA-core kernel)
  *   combine: merges the partials of split rows into u/lse */
 mla_status mla_decode_plan(const mla_decode_params* p, void* workspace, size_t workspace_bytes,
                            void* stream);
@@ -209,6 +210,27 @@ mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_c
  */
 mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c,
                        int d_v, mla_dtype dtype, void* stream);
+
+/*
+ * Merge of partial decode results over disjoint parts of the same query
+ * rows' context ("MLA deep compression", absorption section: u is the
+ * softmax-weighted sum over every cached position, so results over pieces of
+ * the context combine by their log-sum-exp):
+ *   lse[row]    = log sum_r exp(lse_parts[r, row])
+ *   u[row, :]   = sum_r exp(lse_parts[r, row] - lse[row]) u_parts[r, row, :]
+ * For context parallelism across GPUs: each GPU decodes a page range of every
+ * sequence with mla_decode (s_q = 1), the (u, lse) of all GPUs are gathered,
+ * and this call merges them on each GPU.
+ *   u_parts    [R, rows, d_c]  device, read  (dtype)
+ *   lse_parts  [R, rows] fp32  device, read; -inf marks a part without tokens
+ *   u          [rows, d_c]     device, written (dtype)
+ *   lse        [rows] fp32     device, written; may be NULL
+ * rows = B * s_q * n_h (the flattened rows of mla_decode's u); R >= 1; d_c a
+ * positive multiple of 8; u_parts, u and lse 16-byte aligned.  A row whose
+ * parts are all -inf gets u = 0 and lse = -inf.  rows = 0 is a no-op.
+ */
+mla_status mla_merge_partials(const void* u_parts, const float* lse_parts, void* u, float* lse,
+                              int R, int rows, int d_c, mla_dtype dtype, void* stream);
 
 /* Synchronizes `stream`, then reads and clears the device flag of the
  * current device.  Returns MLA_OK if no flag was raised, otherwise

@@ -232,6 +232,10 @@ mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s)
 
 }  // namespace
 
+// csrc/merge.cu: the merge of partial results over pieces of the context
+cudaError_t launch_merge(const void* u_parts, const float* lse_parts, void* u, float* lse, int R,
+                         int rows, int d_c, bool bf16, cudaStream_t s);
+
 WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks) {
   WsLayout L;
   L.slots = (long long)(B + num_chunks) * s_q;
@@ -509,6 +513,23 @@ mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h,
   g.err = d->flags;
   g.bf16 = dtype == MLA_DTYPE_BF16;
   return cuda_status(launch_gemm(g, s));
+}
+
+mla_status mla_merge_partials(const void* u_parts, const float* lse_parts, void* u, float* lse,
+                              int R, int rows, int d_c, mla_dtype dtype, void* stream) {
+  if (!valid_dtype(dtype) || R < 1 || rows < 0 || d_c < 8 || d_c % 8 != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (!u_parts || !lse_parts || !u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(u_parts) || !aligned16(u) || (lse && !aligned16(lse)) ||
+      (reinterpret_cast<uintptr_t>(lse_parts) & 3u) != 0)
+    return MLA_ERR_INVALID_ARG;
+  if ((long long)R * rows * d_c > (1LL << 40)) return MLA_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  return cuda_status(launch_merge(u_parts, lse_parts, u, lse, R, rows, d_c,
+                                  dtype == MLA_DTYPE_BF16, static_cast<cudaStream_t>(stream)));
 }
 
 mla_status mla_check_device_errors(void* stream, int* flags) {

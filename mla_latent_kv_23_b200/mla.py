@@ -55,6 +55,7 @@ SIGNATURES = {
     "mla_decode_kernel_info": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
     "mla_decode_noalloc": ([_P, _V], _I),
     "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _V], _I),
+    "mla_merge_partials": ([_V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
     "mla_check_device_errors": ([_V, ctypes.POINTER(_I)], _I),
 }
 
@@ -211,6 +212,19 @@ def mla_up_proj(u, W_UV, o, stream=None) -> None:
     assert W_UV.shape == (n_h, d_v, d_c) and o.shape == (T, n_h, d_v)
     _check(lib().mla_up_proj(_ptr(u), _ptr(W_UV), _ptr(o), T, n_h, d_c, d_v, _dtype_code(u),
                              _stream(stream)), "mla_up_proj")
+
+
+def mla_merge_partials(u_parts, lse_parts, u, lse=None, stream=None) -> None:
+    """Merge R partial (u, lse) over pieces of the same rows' context:
+    u_parts [R, ..., d_c], lse_parts [R, ...] fp32 -> u [..., d_c], lse [...]."""
+    R = u_parts.shape[0]
+    d_c = u_parts.shape[-1]
+    rows = u.numel() // d_c
+    assert u_parts.numel() == R * rows * d_c and lse_parts.numel() == R * rows
+    assert u_parts.is_contiguous() and lse_parts.is_contiguous() and u.is_contiguous()
+    assert u_parts.dtype == u.dtype and (lse is None or lse.numel() == rows)
+    _check(lib().mla_merge_partials(_ptr(u_parts), _ptr(lse_parts), _ptr(u), _ptr(lse), R, rows,
+                                    d_c, _dtype_code(u), _stream(stream)), "mla_merge_partials")
 
 
 def mla_check_device_errors(stream=None) -> int:

@@ -246,3 +246,71 @@ def test_absorb_and_query_against_oracle():
             for i in (0, 100):
                 qref = orc.absorbed_query(inp, w, b, r, i)
                 assert np.max(np.abs(qd[b, r, i] - qref) / (1 + np.abs(qref))) < 2e-2
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_pieces_decoded_apart_merge_to_the_whole(world):
+    # context parallelism with its ranks emulated as separate decode calls on
+    # one GPU: each call sees one contiguous page range of every sequence;
+    # mla_merge_partials combines the partial (u, lse)
+    from mla_latent_kv_23_b200 import shard
+    w = v3_small(B=3, seqlens=(1000, 777, 4100))
+    inp = synth.draw(w)
+    q = synth.random_q(w)
+    qd, cache = to_dev(q, w), to_dev(inp["cache"], w)
+    us, ls = [], []
+    for pieces in shard.split_context(inp["seqlens"], world, w.page_size):
+        bt, sl = shard.local_tables(inp["block_table"], pieces, w.page_size)
+        u_r, l_r = mla.decode(qd, cache, to_dev_i32(bt), to_dev_i32(sl), w.page_size, w.d_R,
+                              w.softmax_scale)
+        us.append(u_r)
+        ls.append(l_r)
+    u_parts, lse_parts = torch.stack(us).contiguous(), torch.stack(ls).contiguous()
+    u, lse = torch.empty_like(us[0]), torch.empty_like(ls[0])
+    mla.mla_merge_partials(u_parts, lse_parts, u, lse)
+    mla.mla_check_device_errors()
+    picks = [(b, 0, i) for b in range(w.B) for i in (0, 1, 64, 127)]
+    ref = orc.decode_absorbed(q, inp["cache"], inp["block_table"], inp["seqlens"], w, picks)
+    uu, ll = f64(u), f64(lse)
+    for (b, r, i), (u_ref, lse_ref) in ref.items():
+        assert np.max(np.abs(uu[b, r, i] - u_ref) / (1 + np.abs(u_ref))) <= ATOL_REL
+        assert abs(ll[b, r, i] - lse_ref) / max(abs(lse_ref), 1.0) <= 1e-3
+    # and it agrees with one decode of the whole contexts
+    u_full, l_full = mla.decode(qd, cache, to_dev_i32(inp["block_table"]),
+                                to_dev_i32(inp["seqlens"]), w.page_size, w.d_R, w.softmax_scale)
+    assert np.max(np.abs(uu - f64(u_full)) / (1 + np.abs(f64(u_full)))) <= ATOL_REL
+    assert np.max(np.abs(ll - f64(l_full)) / np.maximum(np.abs(f64(l_full)), 1.0)) <= 1e-4
+
+
+@pytest.mark.parametrize("dtype,d_c,R", [(torch.bfloat16, 512, 5), (torch.float32, 64, 3),
+                                         (torch.bfloat16, 264, 40)])
+def test_merge_partials_against_its_definition(dtype, d_c, R):
+    # the merge on its own, against lse = log sum exp, u = sum exp(lse_r - lse) u_r in
+    # fp64 on the same (rounded) inputs; parts marked -inf carry no weight and a
+    # row whose parts are all -inf gives u = 0, lse = -inf
+    g = torch.Generator().manual_seed(3)
+    rows = 37
+    u_parts = torch.randn((R, rows, d_c), generator=g).to(dtype)
+    lse_parts = (torch.randn((R, rows), generator=g) * 20).float()
+    lse_parts[0, 1] = -float("inf")
+    lse_parts[:, 2] = -float("inf")
+    u = torch.empty((rows, d_c), dtype=dtype, device="cuda")
+    lse = torch.empty((rows,), dtype=torch.float32, device="cuda")
+    mla.mla_merge_partials(u_parts.cuda(), lse_parts.cuda(), u, lse)
+    mla.mla_check_device_errors()
+    up, lp = u_parts.double(), lse_parts.double()
+    m = lp.max(dim=0).values
+    ok = torch.isfinite(m)
+    wts = torch.where(torch.isfinite(lp), torch.exp(lp - torch.where(ok, m, 0.0)), 0.0)
+    z = wts.sum(dim=0)
+    lse_ref = torch.where(ok, m + torch.log(torch.where(ok, z, 1.0)), -float("inf"))
+    u_ref = torch.where(ok.unsqueeze(-1),
+                        (wts.unsqueeze(-1) * up).sum(0) / torch.where(ok, z, 1.0).unsqueeze(-1), 0.0)
+    got_u, got_l = u.double().cpu(), lse.double().cpu()
+    assert torch.all(got_u[2] == 0) and got_l[2] == -float("inf")
+    fin = ok.clone()
+    assert torch.allclose(got_l[fin], lse_ref[fin], rtol=1e-6, atol=1e-5)
+    # fp32 weights and sums, bf16 (2^-9) or fp32 output rounding
+    tol = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
+    err = (got_u[fin] - u_ref[fin]).abs() / (1 + u_ref[fin].abs())
+    assert err.max() <= tol
