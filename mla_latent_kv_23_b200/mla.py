@@ -103,6 +103,10 @@ def _dtype_code(t) -> int:
 def _ptr(t) -> Optional[int]:
     if t is None:
         return None
+    if not t.is_cuda:
+        # the library's kernels read and write device memory only; a host
+        # pointer would fault on the GPU
+        raise ValueError("tensors must be on a CUDA device")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return t.data_ptr()

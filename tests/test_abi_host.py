@@ -92,3 +92,12 @@ def test_other_entry_points_reject_bad_arguments(lib):
                                  None) == INVALID
     assert lib.mla_append_latent(16, 32, 48, 64, 80, 96, 4, 64, 8, None, 4, 256, 64, 16, 1e4, 0,
                                  None) == INVALID
+
+
+def test_binding_refuses_host_tensors():
+    # the kernels read device memory only: host tensors never reach the library
+    import torch
+    t = torch.zeros(16)
+    with pytest.raises(ValueError):
+        mla._ptr(t)
+    assert mla._ptr(None) is None
