@@ -101,3 +101,22 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError):
         mla._ptr(t)
     assert mla._ptr(None) is None
+
+
+@pytest.mark.parametrize("args,want", [
+    ((16, 32, 48, 64, 0, 10, 512, 0), INVALID),        # R = 0
+    ((16, 32, 48, 64, 2, -1, 512, 0), INVALID),        # rows < 0
+    ((16, 32, 48, 64, 2, 10, 12, 0), INVALID),         # d_c not a multiple of 8
+    ((16, 32, 48, 64, 2, 10, 0, 0), INVALID),          # d_c = 0
+    ((16, 32, 48, 64, 2, 10, 512, 7), INVALID),        # dtype
+    ((None, 32, 48, 64, 2, 10, 512, 0), INVALID),      # u_parts
+    ((16, None, 48, 64, 2, 10, 512, 0), INVALID),      # lse_parts
+    ((16, 32, None, 64, 2, 10, 512, 0), INVALID),      # u
+    ((17, 32, 48, 64, 2, 10, 512, 0), INVALID),        # u_parts not 16-byte aligned
+    ((16, 34, 48, 64, 2, 10, 512, 0), INVALID),        # lse_parts not 4-byte aligned
+    ((16, 32, 48, 68, 2, 10, 512, 0), INVALID),        # lse not 16-byte aligned
+    ((None, None, None, None, 3, 0, 512, 0), OK),      # rows = 0: nothing to do
+])
+def test_merge_rejects_bad_arguments(lib, args, want):
+    u_parts, lse_parts, u, lse, R, rows, d_c, dt = args
+    assert lib.mla_merge_partials(u_parts, lse_parts, u, lse, R, rows, d_c, dt, None) == want
