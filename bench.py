@@ -252,8 +252,8 @@ def run_gpu(args, w):
     wr = w.with_(seed=w.seed + 1000 * rank) if rank else w
     inp = synth.draw(wr)
     tdt = torch.bfloat16
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from gpu_pipeline import absorb_and_query
+    udt = torch.float32 if args.u_dtype == "fp32" else torch.bfloat16
+    from mla_latent_kv_23_b200.device_inputs import absorb_and_query
     q0, W_QK = absorb_and_query(wr, inp, dev)
     del W_QK
     cache_bytes = inp["num_pages"] * w.page_size * w.width * 2
@@ -267,7 +267,7 @@ def run_gpu(args, w):
     sl = torch.from_numpy(inp["seqlens"]).to(dev)
     W_UV = torch.from_numpy(inp["W_UV"]).to(dev).to(tdt)
     T = w.B * w.s_q
-    u = torch.empty((w.B, w.s_q, w.n_h, w.d_c), dtype=tdt, device=dev)
+    u = torch.empty((w.B, w.s_q, w.n_h, w.d_c), dtype=udt, device=dev)
     lse = torch.empty((w.B, w.s_q, w.n_h), dtype=torch.float32, device=dev)
     o = torch.empty((T, w.n_h, w.d_v), dtype=tdt, device=dev)
     params = [mla.decode_params(qs[i], caches[i], bt, sl, u, lse, w.page_size, w.d_R,
@@ -278,14 +278,19 @@ def run_gpu(args, w):
         raise RuntimeError("the tensor-core decode kernel was not selected for this workload")
 
     def step(i, ev=None):
+        # the caller's step: mla_decode (plan, attend and combine chained by
+        # programmatic dependent launch) and the up-projection; with events,
+        # the stages are called one by one so that the attend kernel alone
+        # sits between the two event nodes
         p = params[i % R]
-        mla.mla_decode_plan(p, ws)
-        if ev is not None:
+        if ev is None:
+            mla.mla_decode(p, ws)
+        else:
+            mla.mla_decode_plan(p, ws)
             ev[0].record()
-        mla.mla_decode_attend(p, ws)
-        if ev is not None:
+            mla.mla_decode_attend(p, ws)
             ev[1].record()
-        mla.mla_decode_combine(p, ws)
+            mla.mla_decode_combine(p, ws)
         mla.mla_up_proj(u.view(T, w.n_h, w.d_c), W_UV, o)
 
     # direct launches once (initialises the library, checks flags)
@@ -437,7 +442,8 @@ def run_e2e(args, w, inp, q0, bt, sl, W_UV, dev, stream, mla, step_flops, world)
     d_q = torch.empty(h_q.shape, dtype=tdt, device=dev)
     d_bt = torch.empty(h_bt.shape, dtype=torch.int32, device=dev)
     d_sl = torch.empty(h_sl.shape, dtype=torch.int32, device=dev)
-    u = torch.empty((w.B, w.s_q, w.n_h, w.d_c), dtype=tdt, device=dev)
+    u = torch.empty((w.B, w.s_q, w.n_h, w.d_c), dtype=torch.float32 if args.u_dtype == "fp32"
+                    else tdt, device=dev)
     lse = torch.empty((w.B, w.s_q, w.n_h), dtype=torch.float32, device=dev)
     o = torch.empty((T, w.n_h, w.d_v), dtype=tdt, device=dev)
     p = mla.decode_params(d_q, d_cache, d_bt, d_sl, u, lse, w.page_size, w.d_R, w.softmax_scale)
@@ -491,6 +497,9 @@ def main():
                     help="host time for the oracle baseline (0 = skip)")
     ap.add_argument("--e2e-steps", type=int, default=20,
                     help="steps of the end-to-end (host buffers) measurement (0 = skip)")
+    ap.add_argument("--u-dtype", default="fp32", choices=["fp32", "bf16"],
+                    help="type of the decode's u (fp32: the precision the parity tests hold "
+                         "every workload to)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -129,7 +129,7 @@ typedef struct {
   const void* kv_cache;     /* [num_pages * page_size, d_c + d_R] device; row = c || k^R        */
   const int* block_table;   /* [B, max_pages_per_seq] int32 device; physical page ids          */
   const int* seqlens;       /* [B] int32 device; cached tokens incl. the s_q query tokens        */
-  void* u;                  /* [B, s_q, n_h, d_c] device, written                                */
+  void* u;                  /* [B, s_q, n_h, d_c] device, written; bf16 or fp32 (see u_fp32)     */
   float* lse;               /* [B, s_q, n_h] fp32 device, written; may be NULL                   */
   int B;                    /* sequences; 0 is a no-op                                           */
   int s_q;                  /* query rows per sequence: 1 or 2                                   */
@@ -142,6 +142,13 @@ typedef struct {
   float softmax_scale;      /* multiplies the scores before softmax, finite and > 0               */
   mla_dtype dtype;          /* of q, kv_cache and u                                              */
   int num_splits;           /* KV chunks the whole batch is cut into; 0 = one per SM pair        */
+  int u_fp32;               /* nonzero: u (and the partial results of split rows) are fp32;
+                               0: u has type `dtype`.  With bf16 inputs an fp32 u carries the
+                               softmax-weighted latent sum to the up-projection unrounded: a
+                               bf16 u moves o = W_UV u by up to 2^-8 |u| per element, which for
+                               contexts dominated by a few large latents (|u| ~ 25) exceeds an
+                               elementwise 2e-2 (1 + |o|) budget where o is near zero.  fp32
+                               inputs always give an fp32 u.                                    */
 } mla_decode_params;
 
 /* Bytes of device scratch mla_decode needs for these parameters (depends on
@@ -160,9 +167,11 @@ mla_status mla_decode(const mla_decode_params* p, void* workspace, size_t worksp
  * separately; calling them in this order is exactly mla_decode.
  *   plan:    per-sequence tile counts and KV-chunk boundaries into the workspace
  *   attend:  the chunked attention (writes u/lse directly for unsplit rows,
- *            partials into the workspace otherwise: bf16 from the
- *            tensor-core kernel, fp32 from the CUDA-core kernel)
- *   combine: merges the partials of split rows into u/lse */
+ *            partials into the workspace otherwise, in the type of u)
+ *   combine: merges the partials of split rows into u/lse
+ * Called on their own, the stages launch as plain stream-ordered kernels;
+ * inside mla_decode each stage may start its prologue while the previous
+ * one finishes (programmatic dependent launch). */
 mla_status mla_decode_plan(const mla_decode_params* p, void* workspace, size_t workspace_bytes,
                            void* stream);
 mla_status mla_decode_attend(const mla_decode_params* p, void* workspace, size_t workspace_bytes,
@@ -199,17 +208,18 @@ mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_c
 /*
  * Per-head up-projection ("MLA deep compression", absorption section, output
  * equation):  o[t, i, :] = W_UV[i] . u[t, i, :]
- *   u     [T, n_h, d_c]   device, read   (T = B * s_q)
- *   W_UV  [n_h, d_v, d_c] device, read
- *   o     [T, n_h, d_v]   device, written
- * The bf16 tensor-core kernel (d_v = 128, d_c a multiple of 64 up to 512)
- * starts reading W_UV before the previous kernel on the stream has finished
- * (programmatic dependent launch; u is read only after it has).  So W_UV
- * must not be written by the kernel launched immediately before this call
- * on the same stream; weights written earlier, or by a copy, are fine.
+ *   u     [T, n_h, d_c]   device, read   (T = B * s_q), type u_dtype
+ *   W_UV  [n_h, d_v, d_c] device, read,    type dtype
+ *   o     [T, n_h, d_v]   device, written, type dtype
+ * Runs on the tensor cores: bf16 weights with a bf16 u, or with an fp32 u
+ * split into two bf16 terms (u = hi + lo, |u - hi - lo| <= 2^-16 |u|) whose
+ * products are accumulated together, so an fp32 u is used to well below
+ * bf16 rounding; fp32 weights (and then an fp32 u) run as tf32.  Supported:
+ * d_v <= 128, d_c a multiple of 64 (bf16) or 32 (fp32) up to 512.
+ * u_dtype must be dtype or MLA_DTYPE_FP32.
  */
 mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c,
-                       int d_v, mla_dtype dtype, void* stream);
+                       int d_v, mla_dtype u_dtype, mla_dtype dtype, void* stream);
 
 /*
  * Merge of partial decode results over disjoint parts of the same query

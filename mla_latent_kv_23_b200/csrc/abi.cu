@@ -169,8 +169,10 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   a.num_chunks = G;
   a.scale = p->softmax_scale;
   a.bf16 = p->dtype == MLA_DTYPE_BF16;
+  a.out_f32 = p->u_fp32 != 0 || p->dtype == MLA_DTYPE_FP32;
   r->tc = use_tensor_cores(p, r->dev);
-  a.part_bf16 = r->tc;
+  a.part_bf16 = r->tc && !a.out_f32;
+  a.pdl = false;
   return MLA_OK;
 }
 
@@ -199,20 +201,27 @@ mla_status encode_q(CUtensorMap* m, const void* ptr, uint64_t n_h, uint64_t qrow
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// 3D map over an output [rows, n_h, 512] (bf16) for TMA stores: box 64 x 32
-// heads x 1, 128-byte swizzle.
-mla_status encode_out(CUtensorMap* m, void* ptr, uint64_t n_h, uint64_t rows) {
+// 3D map over an output [rows, n_h, 512] for TMA stores, 128-byte swizzle:
+// bf16 with boxes of 64 columns x 32 heads x 1, or fp32 with boxes of 32
+// columns x 32 heads x 1 (one 128-byte line per head either way).
+mla_status encode_out(CUtensorMap* m, void* ptr, uint64_t n_h, uint64_t rows, bool f32) {
+  const uint64_t es = f32 ? 4 : 2;
   const cuuint64_t dims[3] = {512, n_h, rows};
-  const cuuint64_t strides[2] = {512 * 2, n_h * 512 * 2};
-  const cuuint32_t box[3] = {64, 32, 1};
+  const cuuint64_t strides[2] = {512 * es, n_h * 512 * es};
+  const cuuint32_t box[3] = {f32 ? 32u : 64u, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+  CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        3, ptr, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s) {
+// Called on its own (pdl = false) a stage is a plain stream-ordered launch;
+// inside mla_decode the attend and combine stages may start their prologues
+// while the previous stage finishes.
+mla_status attend(Resolved r, const mla_decode_params* p, cudaStream_t s, bool pdl) {
+  r.a.pdl = pdl;
   if (!r.tc) return cuda_status(launch_decode_simt(r.a, s));
   Sm100Maps maps;
   const uint64_t kvrows = (uint64_t)p->num_pages * p->page_size;
@@ -224,8 +233,9 @@ mla_status attend(const Resolved& r, const mla_decode_params* p, cudaStream_t s)
   if ((st = encode_q(&maps.q_lat, p->q, p->n_h, qrows, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
       (st = encode_q(&maps.q_rope, p->q, p->n_h, qrows, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
     return st;
-  if ((st = encode_out(&maps.u_out, p->u, p->n_h, qrows)) != MLA_OK ||
-      (st = encode_out(&maps.part_out, r.a.part_u, p->n_h, (uint64_t)r.slots)) != MLA_OK)
+  if ((st = encode_out(&maps.u_out, p->u, p->n_h, qrows, r.a.out_f32)) != MLA_OK ||
+      (st = encode_out(&maps.part_out, r.a.part_u, p->n_h, (uint64_t)r.slots, r.a.out_f32)) !=
+          MLA_OK)
     return st;
   return cuda_status(launch_decode_sm100(r.a, maps, s));
 }
@@ -310,7 +320,7 @@ mla_status mla_decode_attend(const mla_decode_params* p, void* ws, size_t ws_byt
   Resolved r;
   mla_status st = resolve(p, ws, ws_bytes, &r);
   if (st != MLA_OK) return st;
-  return attend(r, p, static_cast<cudaStream_t>(stream));
+  return attend(r, p, static_cast<cudaStream_t>(stream), false);
 }
 
 mla_status mla_decode_combine(const mla_decode_params* p, void* ws, size_t ws_bytes, void* stream) {
@@ -328,7 +338,8 @@ mla_status mla_decode(const mla_decode_params* p, void* ws, size_t ws_bytes, voi
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
-  if ((st = attend(r, p, s)) != MLA_OK) return st;
+  if ((st = attend(r, p, s, true)) != MLA_OK) return st;
+  r.a.pdl = true;
   return cuda_status(launch_combine(r.a, s));
 }
 
@@ -467,52 +478,51 @@ mla_status mla_append_latent(const void* h, const void* W_DKV, const void* W_KR,
 }
 
 mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c, int d_v,
-                       mla_dtype dtype, void* stream) {
-  if (!valid_dtype(dtype) || T < 0 || n_h < 1 || d_c < 1 || d_v < 1) return MLA_ERR_INVALID_ARG;
+                       mla_dtype u_dtype, mla_dtype dtype, void* stream) {
+  if (!valid_dtype(dtype) || !valid_dtype(u_dtype) || T < 0 || n_h < 1 || d_c < 1 || d_v < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (u_dtype != dtype && u_dtype != MLA_DTYPE_FP32) return MLA_ERR_INVALID_ARG;
   if (T == 0) return MLA_OK;
   if (!u || !W_UV || !o) return MLA_ERR_INVALID_ARG;
   if (!aligned16(u) || !aligned16(W_UV) || !aligned16(o)) return MLA_ERR_INVALID_ARG;
-  if (n_h > 65535 || T > 65535 * 64) return MLA_ERR_UNSUPPORTED;
+  if (n_h > 65535 || T > 65535 * 32 || d_v > 128) return MLA_ERR_UNSUPPORTED;
+  const bool f32 = dtype == MLA_DTYPE_FP32;
+  if (f32 ? (d_c % 32 != 0 || d_c > 256) : (d_c % 64 != 0 || d_c > 512))
+    return MLA_ERR_UNSUPPORTED;
+  if ((long long)n_h * d_v > INT_MAX) return MLA_ERR_UNSUPPORTED;
   const DeviceInfo* d = nullptr;
   mla_status st = device_info(&d);
   if (st != MLA_OK) return st;
+  if (!d->up_proj_tc || g_encode == nullptr) return MLA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->up_proj_tc && g_encode != nullptr && dtype == MLA_DTYPE_BF16 && d_v == 128 &&
-      d_c % 64 == 0 && d_c <= 512) {
-    CUtensorMap w_map, u_map;
-    if ((st = encode_2d(&w_map, W_UV, d_c, (uint64_t)n_h * d_v, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-      return st;
-    const cuuint64_t dims[3] = {(cuuint64_t)d_c, (cuuint64_t)n_h, (cuuint64_t)T};
-    const cuuint64_t strides[2] = {(cuuint64_t)d_c * 2, (cuuint64_t)n_h * d_c * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)up_proj_sm100_box_rows(T)};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    if (g_encode(&u_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(u), dims, strides,
-                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const uint64_t es = f32 ? 4 : 2;
+  const CUtensorMapDataType tdt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint32_t cols = static_cast<cuuint32_t>(128 / es);  // one 128-byte row per box row
+  CUtensorMap w_map, u_map;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)d_c, (cuuint64_t)n_h * d_v};
+    const cuuint64_t strides[1] = {(cuuint64_t)d_c * es};
+    const cuuint32_t box[2] = {cols, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    if (g_encode(&w_map, tdt, 2, const_cast<void*>(W_UV), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MLA_ERR_CUDA;
-    return cuda_status(launch_up_proj_sm100(w_map, u_map, o, d->flags, T, n_h, d_c, s));
   }
-  GemmArgs g = {};
-  g.A = u;     // A(z = head, m = t, k = c) = u[t][z][c]
-  g.Bm = W_UV; // B(z, n = v, k = c) = W_UV[z][v][c]
-  g.C = o;     // C(z, m = t, n = v) = o[t][z][v]
-  g.M = T;
-  g.N = d_v;
-  g.K = d_c;
-  g.Z = n_h;
-  g.sAz = d_c;
-  g.sAm = (long long)n_h * d_c;
-  g.sAk = 1;
-  g.sBz = (long long)d_v * d_c;
-  g.sBn = d_c;
-  g.sBk = 1;
-  g.sCz = d_v;
-  g.sCm = (long long)n_h * d_v;
-  g.seg = INT_MAX;
-  g.err = d->flags;
-  g.bf16 = dtype == MLA_DTYPE_BF16;
-  return cuda_status(launch_gemm(g, s));
+  if (!f32 && u_dtype == MLA_DTYPE_FP32)
+    return cuda_status(launch_up_proj_sm100_f32u(w_map, static_cast<const float*>(u), o, d->flags,
+                                                 T, n_h, d_c, d_v, false, s));
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)d_c, (cuuint64_t)n_h, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)d_c * es, (cuuint64_t)n_h * d_c * es};
+    const cuuint32_t box[3] = {cols, 1, (cuuint32_t)up_proj_sm100_box_rows(T)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (g_encode(&u_map, tdt, 3, const_cast<void*>(u), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  return cuda_status(launch_up_proj_sm100(w_map, u_map, o, d->flags, T, n_h, d_c, d_v, f32, false, s));
 }
 
 mla_status mla_merge_partials(const void* u_parts, const float* lse_parts, void* u, float* lse,

@@ -22,7 +22,7 @@ __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162
 __device__ __forceinline__ void st(float* p, float v) { *p = v; }
 __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-template <typename T>
+template <typename T, typename U>
 __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs a) {
   extern __shared__ float sm[];
   const int W = a.d_c + a.d_R;
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
     const float lse = l > 0.f ? m + logf(l) : -INFINITY;
     const size_t orow = (size_t)(b * a.s_q + r) * a.n_h + h;
     if (sg.whole) {
-      T* u = static_cast<T*>(a.u) + orow * a.d_c;
+      U* u = static_cast<U*>(a.u) + orow * a.d_c;
 #pragma unroll
       for (int k = 0; k < kColsPerThread; ++k) {
         const int c = tid + k * kThreads;
@@ -125,10 +125,12 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeArgs 
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s) {
   dim3 grid(a.num_chunks * a.s_q, a.n_h);
   const size_t smem = (size_t)(a.d_c + a.d_R + kTileTokens) * sizeof(float);
-  if (a.bf16)
-    decode_simt_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
+  if (a.bf16 && !a.out_f32)
+    decode_simt_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
+  else if (a.bf16)
+    decode_simt_kernel<__nv_bfloat16, float><<<grid, kThreads, smem, s>>>(a);
   else
-    decode_simt_kernel<float><<<grid, kThreads, smem, s>>>(a);
+    decode_simt_kernel<float, float><<<grid, kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 

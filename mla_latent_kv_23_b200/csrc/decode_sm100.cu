@@ -149,6 +149,7 @@ struct Params {
   float* lse;
   int* err;
   int B, s_q, n_h, max_pages, page_size, num_pages;
+  int out_f32;       // u and the split partials are fp32 (else bf16)
   float scale_log2;  // softmax_scale * log2(e)
 };
 
@@ -673,41 +674,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
       const int col0 = 256 * c + 128 * (qd >> 1);  // latent column of TMEM column kTmemO + 128c
       // The segment's last S has read Q, so the query area stages the output:
-      // 8 KB per warp, its 32 heads x 128 columns as two boxes of 64 columns
-      // in the 128-byte-swizzled layout of the output tensor map (row = head =
-      // lane, 16-byte chunk k of a row at k ^ (row & 7)).  Each box leaves by
-      // one TMA store, which writes whole 128-byte lines of u; the relay loads
-      // the next segment's query only after the stores have read the area.
+      // 8 KB per warp, its 32 heads x 128 columns as boxes of 128-byte lines
+      // (64 bf16 or 32 fp32 columns) in the 128-byte-swizzled layout of the
+      // output tensor map (row = head = lane, 16-byte chunk k of a row at
+      // k ^ (row & 7)).  Each box leaves by one TMA store, which writes whole
+      // 128-byte lines of u; the relay loads the next segment's query only
+      // after the stores have read the area.
       const uint32_t stg = sbase + kOffQ + sw_warp * 8192u;
       const int y_head = 64 * (int)rank + 32 * (qd & 1);  // first head of this warp's rows
       const CUtensorMap* omap = sg.whole ? &p.maps.u_out : &p.maps.part_out;
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
-        tmem_wait_ld();
-        // u of a whole sequence, or this segment's partial u (the combine
-        // stage weights and sums the partials in fp32): bf16 either way
-        const uint32_t row = stg + static_cast<uint32_t>(c0 >> 6) * 4096u + lane * 128u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint32_t w[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const __nv_bfloat162 h2 =
-                __floats2bfloat162_rn(o[8 * e + 2 * k] * inv, o[8 * e + 2 * k + 1] * inv);
-            w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+      if (p.out_f32) {
+        // fp32: four boxes of 32 columns (one 128-byte line per head), two
+        // at a time through the warp's 8 KB
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
+          tmem_wait_ld();
+          const uint32_t box = stg + static_cast<uint32_t>((c0 >> 5) & 1) * 4096u;
+          if (c0 == 64) {  // the first two boxes must have left before reuse
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
           }
-          const uint32_t chunk16 = static_cast<uint32_t>(((c0 & 63) >> 3) + e);
-          st_shared_v4(row + ((chunk16 ^ static_cast<uint32_t>(lane & 7)) << 4), w[0], w[1], w[2],
-                       w[3]);
-        }
-        if (c0 & 32) {  // box c0 >> 6 is complete
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            st_shared_v4(box + lane * 128u + ((static_cast<uint32_t>(e ^ (lane & 7))) << 4),
+                         __float_as_uint(o[4 * e] * inv), __float_as_uint(o[4 * e + 1] * inv),
+                         __float_as_uint(o[4 * e + 2] * inv), __float_as_uint(o[4 * e + 3] * inv));
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && y_head < p.n_h) {
-            tma_store_3d(omap, stg + static_cast<uint32_t>(c0 >> 6) * 4096u, col0 + (c0 & 64),
-                         y_head, out_z);
+            tma_store_3d(omap, box, col0 + c0, y_head, out_z);
             bulk_commit();
+          }
+        }
+      } else {
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
+          tmem_wait_ld();
+          // u of a whole sequence, or this segment's partial u (the combine
+          // stage weights and sums the partials in fp32): bf16 either way
+          const uint32_t row = stg + static_cast<uint32_t>(c0 >> 6) * 4096u + lane * 128u;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const __nv_bfloat162 h2 =
+                  __floats2bfloat162_rn(o[8 * e + 2 * k] * inv, o[8 * e + 2 * k + 1] * inv);
+              w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            const uint32_t chunk16 = static_cast<uint32_t>(((c0 & 63) >> 3) + e);
+            st_shared_v4(row + ((chunk16 ^ static_cast<uint32_t>(lane & 7)) << 4), w[0], w[1],
+                         w[2], w[3]);
+          }
+          if (c0 & 32) {  // box c0 >> 6 is complete
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && y_head < p.n_h) {
+              tma_store_3d(omap, stg + static_cast<uint32_t>(c0 >> 6) * 4096u, col0 + (c0 & 64),
+                           y_head, out_z);
+              bulk_commit();
+            }
           }
         }
       }
@@ -797,6 +825,7 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   p.max_pages = a.max_pages;
   p.page_size = a.page_size;
   p.num_pages = a.num_pages;
+  p.out_f32 = a.out_f32 ? 1 : 0;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.num_chunks * a.s_q, 1, 1);
@@ -807,7 +836,7 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, decode_sm100_kernel, p);
 }
 

@@ -49,8 +49,10 @@ struct DecodeArgs {
   int* err;
   int B, s_q, n_h, d_c, d_R, page_size, max_pages, num_pages, num_chunks;
   float scale;
-  bool bf16;
-  bool part_bf16;  // split partials of u are stored as bf16 (tensor-core path) instead of fp32
+  bool bf16;       // q and the cache are bf16 (else fp32)
+  bool out_f32;    // u is fp32 (else bf16)
+  bool part_bf16;  // split partials of u are bf16 (exactly when u is bf16)
+  bool pdl;        // launch as a programmatic dependent of the previous kernel
 };
 
 cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s);
@@ -64,8 +66,9 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s);
 // swizzle), RoPE boxes 32 x 16 heads x 1 (64-byte swizzle); heads past n_h
 // read as zero.
 // out maps over u [B * s_q, n_h, 512] and over the split partials
-// [slots, n_h, 512] (bf16): boxes 64 x 32 heads x 1, 128-byte swizzle, for
-// the TMA stores of the epilogue; heads past n_h are not written.
+// [slots, n_h, 512], both bf16 (boxes 64 x 32 heads x 1) or both fp32
+// (boxes 32 x 32 heads x 1), 128-byte swizzle, for the TMA stores of the
+// epilogue; heads past n_h are not written.
 struct Sm100Maps {
   CUtensorMap kv_lat, kv_rope, q_lat, q_rope, u_out, part_out;
 };
@@ -101,13 +104,20 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
-// Per-head up-projection on the tensor cores (bf16, d_v = 128, d_c a
-// multiple of 64 up to 512).  w_map: W_UV as [n_h * 128, d_c], box 64 x 128,
-// 128-byte swizzle; u_map: u as [T, n_h, d_c], box 64 x 1 x
-// up_proj_sm100_box_rows(T), 128-byte swizzle.
+// Per-head up-projection on the tensor cores, d_v <= 128.  w_map: W_UV as
+// [n_h * d_v, d_c] with 128-byte boxes x 128 rows, 128-byte swizzle (bf16:
+// 64 columns; fp32: 32 columns).  u_map: u as [T, n_h, d_c], 128-byte boxes
+// x 1 x up_proj_sm100_box_rows(T), 128-byte swizzle.  f32: W, u and o are
+// fp32 (tf32 MMAs, d_c a multiple of 32 up to 256); else bf16 (d_c a
+// multiple of 64 up to 512).
 int up_proj_sm100_prepare();
 int up_proj_sm100_box_rows(int T);
 cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_map, void* o,
-                                 int* err, int T, int n_h, int d_c, cudaStream_t s);
+                                 int* err, int T, int n_h, int d_c, int d_v, bool f32, bool pdl,
+                                 cudaStream_t s);
+// bf16 W and o with an fp32 u, read with plain loads and split into two bf16
+// terms, u = hi + lo, in shared memory: o = W^UV hi + W^UV lo.
+cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, void* o, int* err,
+                                      int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s);
 
 }  // namespace mla

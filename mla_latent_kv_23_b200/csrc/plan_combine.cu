@@ -223,17 +223,20 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (lse_out != nullptr && lane == 0) lse_out[static_cast<size_t>(br) * n_h + h] = lse_all;
 }
 
-// Merge of bf16 partials with d_c = 512 (the tensor-core path).  One warp per
-// output row; lane l owns columns [16 l, 16 l + 16).  The partials of up to 8
-// splits are loaded before any is used, so a row waits for memory about once
-// per 8 splits instead of once per split.
-template <bool kBf16>
+// Merge of the partials with d_c = 512 (the tensor-core path): bf16 or fp32
+// partials, bf16 or fp32 u.  One warp per output row; lane l owns columns
+// [16 l, 16 l + 16).  The partials of up to kGroup splits (8 bf16 or 4 fp32
+// rows: 32 or 64 bytes per lane each) are loaded before any is used, so a
+// row waits for memory about once per group instead of once per split.
+template <bool kOutBf16, bool kPartBf16>
 __global__ void __launch_bounds__(kCombineThreads)
     combine512_kernel(const int* __restrict__ tile_prefix, const int* __restrict__ split_base,
-                      const __nv_bfloat16* __restrict__ part_u, const float* __restrict__ part_lse,
+                      const void* __restrict__ part_u, const float* __restrict__ part_lse,
                       void* __restrict__ u_out, float* __restrict__ lse_out, int s_q, int n_h,
                       int rows) {
   constexpr int kDc = 512;
+  constexpr int kGroup = kPartBf16 ? 8 : 4;
+  constexpr int kVecs = kPartBf16 ? 2 : 4;  // 16-byte loads per lane per partial row
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   // The plan stage's outputs are read before waiting: that stage completed
@@ -258,20 +261,22 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (nsplit == 0 && tp1 != tp0) return;  // written directly by the attend stage
   const size_t slot0 = static_cast<size_t>(sb0) * s_q + r;  // slot of split s: slot0 + s*s_q
   auto lse_of = [&](int s) { return part_lse[(slot0 + (size_t)s * s_q) * n_h + h]; };
-  auto load_group = [&](int s0, uint4 (&v)[8][2]) {
+  auto load_group = [&](int s0, uint4 (&v)[kGroup][kVecs]) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kGroup; ++k) {
       if (s0 + k < nsplit) {
-        const __nv_bfloat16* src =
-            part_u + ((slot0 + (size_t)(s0 + k) * s_q) * n_h + h) * kDc + 16 * lane;
-        v[k][0] = *reinterpret_cast<const uint4*>(src);
-        v[k][1] = *reinterpret_cast<const uint4*>(src + 8);
+        const size_t e0 = ((slot0 + (size_t)(s0 + k) * s_q) * n_h + h) * kDc + 16 * lane;
+        const uint4* src = kPartBf16
+            ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(part_u) + e0)
+            : reinterpret_cast<const uint4*>(static_cast<const float*>(part_u) + e0);
+#pragma unroll
+        for (int i = 0; i < kVecs; ++i) v[k][i] = src[i];
       }
     }
   };
-  // the first 8 partial rows are requested together with the statistics, so
-  // one memory round trip covers rows with up to 8 pieces
-  uint4 v[8][2];
+  // the first group of partial rows is requested together with the
+  // statistics, so one memory round trip covers rows with few pieces
+  uint4 v[kGroup][kVecs];
   load_group(0, v);
   // one pass: per-lane running (max, sum of exp), then the warp's
   float m = -INFINITY, z = 0.f;
@@ -291,27 +296,33 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   if (m_all != -INFINITY) {
-    for (int s0 = 0; s0 < nsplit; s0 += 8) {
+    for (int s0 = 0; s0 < nsplit; s0 += kGroup) {
       if (s0 > 0) load_group(s0, v);
-      const int n_here = min(8, nsplit - s0);
+      const int n_here = min(kGroup, nsplit - s0);
       const float w_me = lane < n_here ? expf(lse_of(s0 + lane) - lse_all) : 0.f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kGroup; ++k) {
         const float w = __shfl_sync(0xffffffffu, w_me, k);
         if (k < n_here) {
-          const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(v[k]);
+          if (kPartBf16) {
+            const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(v[k]);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 f = __bfloat1622float2(x[e]);
-            acc[2 * e] += w * f.x;
-            acc[2 * e + 1] += w * f.y;
+            for (int e = 0; e < 8; ++e) {
+              const float2 f = __bfloat1622float2(x[e]);
+              acc[2 * e] += w * f.x;
+              acc[2 * e + 1] += w * f.y;
+            }
+          } else {
+            const float* x = reinterpret_cast<const float*>(v[k]);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] += w * x[e];
           }
         }
       }
     }
   }
   const size_t orow = static_cast<size_t>(br) * n_h + h;
-  if (kBf16) {
+  if (kOutBf16) {
     uint32_t pk[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -349,23 +360,27 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.pdl ? 1 : 0;
   const int* tp = a.tile_prefix;
   const int* sb = a.split_base;
   const void* pu = a.part_u;
   const float* pl = a.part_lse;
-  if (a.part_bf16 && a.d_c == 512) {
-    const __nv_bfloat16* pb = static_cast<const __nv_bfloat16*>(pu);
-    if (a.bf16)
-      return cudaLaunchKernelEx(&cfg, combine512_kernel<true>, tp, sb, pb, pl, a.u, a.lse, a.s_q,
-                                a.n_h, rows);
-    return cudaLaunchKernelEx(&cfg, combine512_kernel<false>, tp, sb, pb, pl, a.u, a.lse, a.s_q,
-                              a.n_h, rows);
+  const bool out_bf16 = !a.out_f32;
+  if (a.d_c == 512) {
+    if (a.part_bf16)
+      return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, true>, tp, sb, pu, pl, a.u,
+                                           a.lse, a.s_q, a.n_h, rows)
+                      : cudaLaunchKernelEx(&cfg, combine512_kernel<false, true>, tp, sb, pu, pl,
+                                           a.u, a.lse, a.s_q, a.n_h, rows);
+    return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, false>, tp, sb, pu, pl, a.u,
+                                         a.lse, a.s_q, a.n_h, rows)
+                    : cudaLaunchKernelEx(&cfg, combine512_kernel<false, false>, tp, sb, pu, pl, a.u,
+                                         a.lse, a.s_q, a.n_h, rows);
   }
-  if (a.bf16 && a.part_bf16)
+  if (out_bf16 && a.part_bf16)
     return cudaLaunchKernelEx(&cfg, combine_kernel<true, true>, tp, sb, pu, pl, a.u, a.lse, a.s_q,
                               a.n_h, a.d_c, rows);
-  if (a.bf16)
+  if (out_bf16)
     return cudaLaunchKernelEx(&cfg, combine_kernel<true, false>, tp, sb, pu, pl, a.u, a.lse, a.s_q,
                               a.n_h, a.d_c, rows);
   return cudaLaunchKernelEx(&cfg, combine_kernel<false, false>, tp, sb, pu, pl, a.u, a.lse, a.s_q,

@@ -1,15 +1,23 @@
-// Per-head up-projection on the tensor cores (sm_100a), bf16:
+// Per-head up-projection on the tensor cores (sm_100a):
 //     o[t, i, :] = W^UV_i . u[t, i, :]
 // ("MLA deep compression", absorption section, output equation).
 //
-// One CTA per (head i, block of up to 64 query rows t) computes
+// One CTA per (head i, block of query rows t) computes
 // D[v, t] = sum_c W^UV_i[v, c] u[t, i, c] as one tcgen05 MMA chain with
-// M = d_v = 128, N = rows (padded to 16), K = d_c: W^UV_i (128 KB at
-// d_c = 512) is the K-major A operand and the rows of u are the K-major B
-// operand, both staged by TMA with 128-byte swizzle.  The weight read
-// (16.8 MB over all heads, the whole cost of this step) is issued before the
-// kernel waits for the decode that produces u, so with programmatic
-// dependent launch it overlaps the end of the decode.
+// M = 128 (rows v of W^UV_i; rows past d_v belong to the next head or lie
+// past the tensor and are never stored), N = rows (padded to 16), K = d_c.
+// W^UV_i is the K-major A operand and the rows of u the K-major B operand,
+// both in 128-byte-swizzled shared memory.  Three input modes:
+//   kBf16:   bf16 W and u, both staged by TMA (kind::f16);
+//   kSplitU: bf16 W and an fp32 u, read with plain loads and split into two
+//            bf16 terms hi = bf16(u), lo = bf16(u - hi) written in the
+//            swizzled layout; D = W hi + W lo in one accumulator, so u is
+//            used to within 2^-16 of itself (kind::f16);
+//   kTf32:   fp32 W and u staged by TMA, read as tf32 (kind::tf32).
+// The weight read (16.8 MB over all heads at the DeepSeek-V3 shape, the
+// whole cost of this step) is issued before the kernel waits for the
+// previous kernel, so under programmatic dependent launch it overlaps the
+// end of the decode that produces u.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -19,33 +27,49 @@ namespace mla {
 namespace {
 using namespace ptx;
 
+enum class UpMode { kBf16, kSplitU, kTf32 };
+
 constexpr int kThreads = 128;
-constexpr int kDv = 128;         // M
-constexpr int kMaxN = 64;        // query rows per CTA
-constexpr int kMaxKb = 8;        // d_c / 64 <= 8
-constexpr uint32_t kWBlk = 128 * 128;     // 128 rows x 64 cols bf16
-constexpr uint32_t kUBlk = kMaxN * 128;   // up to 64 rows x 64 cols bf16
+constexpr int kM = 128;              // MMA rows: d_v <= 128
+constexpr int kMaxKb = 8;            // 128-byte column blocks of d_c
+constexpr int kMaxRows = 64;         // query rows per CTA (kBf16, kTf32)
+constexpr int kMaxRowsSplit = 32;    // query rows per CTA (kSplitU: hi and lo)
+constexpr uint32_t kWBlk = kM * 128; // 128 rows x 128 bytes
+
+template <UpMode kMode>
+constexpr int max_rows() { return kMode == UpMode::kSplitU ? kMaxRowsSplit : kMaxRows; }
+template <UpMode kMode>
+constexpr uint32_t u_bytes() {  // B operand area (hi and lo for kSplitU)
+  return (kMode == UpMode::kSplitU ? 2u : 1u) * kMaxKb * max_rows<kMode>() * 128u;
+}
+template <UpMode kMode>
+constexpr size_t smem_bytes() { return kMaxKb * kWBlk + u_bytes<kMode>() + 64 + 1024; }
 
 struct Params {
-  CUtensorMap w_map;   // W_UV as [n_h * d_v rows, d_c cols], box 64 x 128
-  CUtensorMap u_map;   // u as [T, n_h, d_c], box 64 x 1 x n_pad
-  __nv_bfloat16* o;
+  CUtensorMap w_map;   // W_UV as [n_h * d_v rows, d_c cols], box (128 bytes) x 128 rows
+  CUtensorMap u_map;   // u as [T, n_h, d_c], box (128 bytes) x 1 x n_pad (kBf16, kTf32)
+  const float* u_f32;  // u (kSplitU)
+  void* o;             // [T, n_h, d_v]: bf16 (kBf16, kSplitU) or fp32 (kTf32)
   int* err;
-  int T, n_h, d_c, n_pad;
+  int T, n_h, d_c, d_v, n_pad;
 };
 
+template <UpMode kMode>
 __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid_constant__ Params p) {
+  constexpr bool kF32 = kMode == UpMode::kTf32;
+  constexpr int kColsPerBlk = kF32 ? 32 : 64;  // elements in one 128-byte row
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (sbase - raw_addr);
-  const int kb_n = p.d_c / 64;
+  const int kb_n = p.d_c / kColsPerBlk;
   const uint32_t off_u = kMaxKb * kWBlk;
-  const uint32_t off_bar = off_u + kMaxKb * kUBlk;
+  const uint32_t off_bar = off_u + u_bytes<kMode>();
   const uint32_t bar_w = sbase + off_bar, bar_u = bar_w + 8, bar_mma = bar_w + 16;
   const uint32_t tmem_slot = bar_w + 24;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.x, t0 = blockIdx.y * kMaxN;
+  const int head = blockIdx.x, t0 = blockIdx.y * max_rows<kMode>();
+  const uint32_t ublk = p.n_pad * 128;  // one 128-byte column block of the B operand
 
   if (threadIdx.x == 0) {
     mbar_init(bar_w, 1);
@@ -64,33 +88,75 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&p.w_map);
-    prefetch_tmap(&p.u_map);
+    if (kMode != UpMode::kSplitU) prefetch_tmap(&p.u_map);
     // the weights do not depend on the previous kernel: fetch them first
     mbar_arrive_expect_tx(bar_w, kb_n * kWBlk);
     for (int kb = 0; kb < kb_n; ++kb)
-      tma_load_2d(sbase + kb * kWBlk, &p.w_map, bar_w, kb * 64, head * kDv);
+      tma_load_2d(sbase + kb * kWBlk, &p.w_map, bar_w, kb * kColsPerBlk, head * p.d_v);
   }
   pdl_wait_previous();
   pdl_launch_dependents();
+  if constexpr (kMode == UpMode::kSplitU) {
+    // u rows -> hi and lo bf16 terms, 8 columns (one 16-byte chunk of each
+    // term) per step, in the 128-byte swizzle the MMA descriptor expects:
+    // chunk k of row t at byte t * 128 + ((k ^ (t & 7)) << 4) of its block;
+    // rows past T are zero
+    const int chunks = p.d_c / 8;
+    for (int unit = threadIdx.x; unit < p.n_pad * chunks; unit += kThreads) {
+      const int t = unit / chunks, c8 = unit % chunks;
+      float v[8];
+      if (t0 + t < p.T) {
+        const float4* src = reinterpret_cast<const float4*>(
+            p.u_f32 + ((size_t)(t0 + t) * p.n_h + head) * p.d_c + 8 * c8);
+        const float4 a = src[0], b = src[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = 0.f;
+      }
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        const float2 hf = __bfloat1622float2(h2);
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * k] - hf.x, v[2 * k + 1] - hf.y);
+        hi[k] = *reinterpret_cast<const uint32_t*>(&h2);
+        lo[k] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+      const int kb = c8 >> 3, k16 = c8 & 7;
+      const uint32_t off = kb * ublk + t * 128 + ((static_cast<uint32_t>(k16 ^ (t & 7))) << 4);
+      st_shared_v4(sbase + off_u + off, hi[0], hi[1], hi[2], hi[3]);
+      st_shared_v4(sbase + off_u + kMaxKb * ublk + off, lo[0], lo[1], lo[2], lo[3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+  }
   bool ok = true;
   if (threadIdx.x == 0) {
-    const uint32_t ublk = p.n_pad * 128;
-    mbar_arrive_expect_tx(bar_u, kb_n * ublk);
-    for (int kb = 0; kb < kb_n; ++kb)
-      tma_load_3d(sbase + off_u + kb * ublk, &p.u_map, bar_u, kb * 64, head, t0);
-    ok = mbar_wait(bar_w, 0, p.err, MLA_DEVFLAG_TIMEOUT) &&
-         mbar_wait(bar_u, 0, p.err, MLA_DEVFLAG_TIMEOUT);
+    if constexpr (kMode != UpMode::kSplitU) {
+      mbar_arrive_expect_tx(bar_u, kb_n * ublk);
+      for (int kb = 0; kb < kb_n; ++kb)
+        tma_load_3d(sbase + off_u + kb * ublk, &p.u_map, bar_u, kb * kColsPerBlk, head, t0);
+      ok = mbar_wait(bar_u, 0, p.err, MLA_DEVFLAG_TIMEOUT);
+    }
+    ok = ok && mbar_wait(bar_w, 0, p.err, MLA_DEVFLAG_TIMEOUT);
     if (ok) {
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16(kDv, p.n_pad, false);
+      const uint32_t idesc = kF32 ? idesc_tf32(kM, p.n_pad, false) : idesc_bf16(kM, p.n_pad, false);
       uint32_t acc = 0;
-      for (int kb = 0; kb < kb_n; ++kb)
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t a = smem_desc(sbase + kb * kWBlk + ks * 32, 16, 1024, kLayoutSW128);
-          const uint64_t b = smem_desc(sbase + off_u + kb * ublk + ks * 32, 16, 1024, kLayoutSW128);
-          umma_f16_ss(tmem, a, b, idesc, acc);
-          acc = 1;
-        }
+      for (int term = 0; term < (kMode == UpMode::kSplitU ? 2 : 1); ++term)
+        for (int kb = 0; kb < kb_n; ++kb)
+          for (int ks = 0; ks < 4; ++ks) {  // 32 bytes of K per instruction
+            const uint64_t a = smem_desc(sbase + kb * kWBlk + ks * 32, 16, 1024, kLayoutSW128);
+            const uint64_t b = smem_desc(sbase + off_u + (term * kMaxKb + kb) * ublk + ks * 32, 16,
+                                         1024, kLayoutSW128);
+            if (kF32)
+              umma_tf32_ss(tmem, a, b, idesc, acc);
+            else
+              umma_f16_ss(tmem, a, b, idesc, acc);
+            acc = 1;
+          }
     }
     umma_commit(bar_mma);
     if (!mbar_wait(bar_mma, 0, p.err, MLA_DEVFLAG_TIMEOUT)) ok = false;
@@ -105,11 +171,18 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
       float d[32];
       tmem_ld32(tmem + lane_base + c0, d);
       tmem_wait_ld();
+      if (v < p.d_v) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int t = t0 + c0 + k;
-        if (c0 + k < p.n_pad && t < p.T)
-          p.o[((size_t)t * p.n_h + head) * kDv + v] = __float2bfloat16_rn(d[k]);
+        for (int k = 0; k < 32; ++k) {
+          const int t = t0 + c0 + k;
+          if (c0 + k < p.n_pad && t < p.T) {
+            const size_t idx = ((size_t)t * p.n_h + head) * p.d_v + v;
+            if (kF32)
+              static_cast<float*>(p.o)[idx] = d[k];
+            else
+              static_cast<__nv_bfloat16*>(p.o)[idx] = __float2bfloat16_rn(d[k]);
+          }
+        }
       }
     }
   }
@@ -121,47 +194,77 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
   }
 }
 
-constexpr size_t kSmemBytes = kMaxKb * kWBlk + kMaxKb * kUBlk + 64 + 1024;
+template <UpMode kMode>
+cudaError_t launch(const Params& p, int n_h, int T, bool pdl, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_h, (T + max_rows<kMode>() - 1) / max_rows<kMode>(), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<kMode>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, up_proj_sm100_kernel<kMode>, p);
+}
+
+int pad_rows(int T, int cap) {
+  const int rows = T < cap ? T : cap;
+  return (rows + 15) / 16 * 16;
+}
 
 }  // namespace
 
 int up_proj_sm100_prepare() {
-  if (cudaFuncSetAttribute(up_proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemBytes) != cudaSuccess) {
+  if (cudaFuncSetAttribute(up_proj_sm100_kernel<UpMode::kBf16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<UpMode::kBf16>()) != cudaSuccess ||
+      cudaFuncSetAttribute(up_proj_sm100_kernel<UpMode::kSplitU>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<UpMode::kSplitU>()) != cudaSuccess ||
+      cudaFuncSetAttribute(up_proj_sm100_kernel<UpMode::kTf32>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<UpMode::kTf32>()) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
   return 1;
 }
 
+int up_proj_sm100_box_rows(int T) { return pad_rows(T, kMaxRows); }
+
 cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_map, void* o,
-                                 int* err, int T, int n_h, int d_c, cudaStream_t s) {
+                                 int* err, int T, int n_h, int d_c, int d_v, bool f32, bool pdl,
+                                 cudaStream_t s) {
   Params p;
   p.w_map = w_map;
   p.u_map = u_map;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.u_f32 = nullptr;
+  p.o = o;
   p.err = err;
   p.T = T;
   p.n_h = n_h;
   p.d_c = d_c;
-  const int rows = T < kMaxN ? T : kMaxN;
-  p.n_pad = (rows + 15) / 16 * 16;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_h, (T + kMaxN - 1) / kMaxN, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, up_proj_sm100_kernel, p);
+  p.d_v = d_v;
+  p.n_pad = pad_rows(T, kMaxRows);
+  return f32 ? launch<UpMode::kTf32>(p, n_h, T, pdl, s) : launch<UpMode::kBf16>(p, n_h, T, pdl, s);
 }
 
-int up_proj_sm100_box_rows(int T) {
-  const int rows = T < kMaxN ? T : kMaxN;
-  return (rows + 15) / 16 * 16;
+cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, void* o, int* err,
+                                      int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s) {
+  Params p;
+  p.w_map = w_map;
+  memset(&p.u_map, 0, sizeof(p.u_map));
+  p.u_f32 = u;
+  p.o = o;
+  p.err = err;
+  p.T = T;
+  p.n_h = n_h;
+  p.d_c = d_c;
+  p.d_v = d_v;
+  p.n_pad = pad_rows(T, kMaxRowsSplit);
+  return launch<UpMode::kSplitU>(p, n_h, T, pdl, s);
 }
 
 }  // namespace mla

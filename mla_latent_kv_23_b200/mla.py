@@ -37,7 +37,7 @@ class DecodeParams(ctypes.Structure):
                 ("d_c", ctypes.c_int), ("d_R", ctypes.c_int), ("page_size", ctypes.c_int),
                 ("max_pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int),
                 ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int),
-                ("num_splits", ctypes.c_int)]
+                ("num_splits", ctypes.c_int), ("u_fp32", ctypes.c_int)]
 
 
 _V, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -54,7 +54,7 @@ SIGNATURES = {
     "mla_decode_combine": ([_P, _V, _S, _V], _I),
     "mla_decode_kernel_info": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
     "mla_decode_noalloc": ([_P, _V], _I),
-    "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _V], _I),
+    "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
     "mla_merge_partials": ([_V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
     "mla_check_device_errors": ([_V, ctypes.POINTER(_I)], _I),
 }
@@ -156,8 +156,14 @@ def decode_params(q, kv_cache, block_table, seqlens, u, lse, page_size: int, d_R
                   softmax_scale: float, num_splits: int = 0) -> DecodeParams:
     """Pack mla_decode_params from tensors: q [B, s_q, n_h, d_c + d_R],
     kv_cache [num_pages * page_size, d_c + d_R], block_table [B, max_pages],
-    seqlens [B], u [B, s_q, n_h, d_c], lse [B, s_q, n_h] or None."""
+    seqlens [B], u [B, s_q, n_h, d_c] (same dtype as q, or float32),
+    lse [B, s_q, n_h] float32 or None."""
+    torch = _torch()
     B, s_q, n_h, W = q.shape
+    if u.dtype != q.dtype and u.dtype != torch.float32:
+        raise TypeError("u must have the dtype of q or be float32")
+    if lse is not None and lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
     d_c = W - d_R
     rows = kv_cache.shape[0]
     return DecodeParams(q=_ptr(q), kv_cache=_ptr(kv_cache), block_table=_ptr(block_table),
@@ -165,7 +171,8 @@ def decode_params(q, kv_cache, block_table, seqlens, u, lse, page_size: int, d_R
                         d_c=d_c, d_R=d_R, page_size=page_size,
                         max_pages_per_seq=block_table.shape[1] if block_table.dim() == 2 else 1,
                         num_pages=max(rows // page_size, 1), softmax_scale=float(softmax_scale),
-                        dtype=_dtype_code(q), num_splits=num_splits)
+                        dtype=_dtype_code(q), num_splits=num_splits,
+                        u_fp32=int(u.dtype == torch.float32))
 
 
 def mla_decode_workspace_size(p: DecodeParams) -> int:
@@ -211,11 +218,15 @@ def mla_decode_noalloc(p: DecodeParams, stream=None) -> None:
 
 
 def mla_up_proj(u, W_UV, o, stream=None) -> None:
+    """o [T, n_h, d_v] = W_UV [n_h, d_v, d_c] . u [T, n_h, d_c]; o has W_UV's
+    dtype, u that dtype or float32."""
     T, n_h, d_c = u.shape
     d_v = W_UV.shape[1]
     assert W_UV.shape == (n_h, d_v, d_c) and o.shape == (T, n_h, d_v)
+    if o.dtype != W_UV.dtype:
+        raise TypeError("o must have the dtype of W_UV")
     _check(lib().mla_up_proj(_ptr(u), _ptr(W_UV), _ptr(o), T, n_h, d_c, d_v, _dtype_code(u),
-                             _stream(stream)), "mla_up_proj")
+                             _dtype_code(W_UV), _stream(stream)), "mla_up_proj")
 
 
 def mla_merge_partials(u_parts, lse_parts, u, lse=None, stream=None) -> None:
@@ -227,6 +238,12 @@ def mla_merge_partials(u_parts, lse_parts, u, lse=None, stream=None) -> None:
     assert u_parts.numel() == R * rows * d_c and lse_parts.numel() == R * rows
     assert u_parts.is_contiguous() and lse_parts.is_contiguous() and u.is_contiguous()
     assert u_parts.dtype == u.dtype and (lse is None or lse.numel() == rows)
+    torch = _torch()
+    # the kernel reads the statistics as fp32 words
+    if lse_parts.dtype != torch.float32 or (lse is not None and lse.dtype != torch.float32):
+        raise TypeError("lse_parts and lse must be float32")
+    if lse is not None and not lse.is_contiguous():
+        raise ValueError("lse must be contiguous")
     _check(lib().mla_merge_partials(_ptr(u_parts), _ptr(lse_parts), _ptr(u), _ptr(lse), R, rows,
                                     d_c, _dtype_code(u), _stream(stream)), "mla_merge_partials")
 
@@ -248,11 +265,13 @@ def mla_status_string(status: int) -> str:
 # convenience: allocate outputs + workspace and run one decode
 # ----------------------------------------------------------------------------
 def decode(q, kv_cache, block_table, seqlens, page_size: int, d_R: int, softmax_scale: float,
-           num_splits: int = 0, with_lse: bool = True, stream=None):
-    """Returns (u [B, s_q, n_h, d_c], lse [B, s_q, n_h] or None)."""
+           num_splits: int = 0, with_lse: bool = True, stream=None, u_dtype=None):
+    """Returns (u [B, s_q, n_h, d_c], lse [B, s_q, n_h] or None); u has
+    u_dtype (default: float32, which keeps the weighted latent sum unrounded
+    for the up-projection)."""
     torch = _torch()
     B, s_q, n_h, W = q.shape
-    u = torch.empty((B, s_q, n_h, W - d_R), dtype=q.dtype, device=q.device)
+    u = torch.empty((B, s_q, n_h, W - d_R), dtype=u_dtype or torch.float32, device=q.device)
     lse = torch.empty((B, s_q, n_h), dtype=torch.float32, device=q.device) if with_lse else None
     p = decode_params(q, kv_cache, block_table, seqlens, u, lse, page_size, d_R, softmax_scale,
                       num_splits)

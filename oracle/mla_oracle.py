@@ -131,7 +131,7 @@ def gather_rows(cache, block_table, page_size: int, b: int, L: int):
     """Logical rows 0..L-1 of sequence b through its block table."""
     j = np.arange(L)
     rows = np.asarray(block_table)[b, j // page_size].astype(np.int64) * page_size + j % page_size
-    return np.asarray(cache, f64)[rows]
+    return np.asarray(np.asarray(cache)[rows], f64)
 
 
 def pipeline_cache(inp: dict, w) -> np.ndarray:
@@ -245,6 +245,46 @@ def decode_absorbed(q: np.ndarray, cache, block_table, seqlens, w, picks=None,
                 d["abs_v"] = a @ np.abs(C @ Wi.T)
             out[(b, r, i)] = d
     return out
+
+
+def absorbed_queries(inp: dict, w, b: int, r: int) -> np.ndarray:
+    """absorbed_query for every head of row (b, r) at once: q^lat_i =
+    W^UK_i^T (W^Q_i h) and q^R_i = RoPE(W^QR_i h, pos), as [n_h, d_c + d_R]."""
+    h = np.asarray(inp["h_q"][b, r], f64)
+    qn = np.einsum("hkd,d->hk", np.asarray(inp["W_Q"], f64), h)            # W^Q_i h
+    qlat = np.einsum("hkc,hk->hc", np.asarray(inp["W_UK"], f64), qn)      # W^UK_i^T (.)
+    pos = int(inp["qpos"][b, r])
+    qr = np.einsum("hkd,d->hk", np.asarray(inp["W_QR"], f64), h)
+    qr = np.stack([rope(x, pos, w.rope_base) for x in qr])
+    return np.concatenate([qlat, qr], axis=1)
+
+
+def decode_absorbed_seq(q_b: np.ndarray, cache, block_table, L: int, b: int, w,
+                        want_abs: bool = False):
+    """decode_absorbed for every query row and head of sequence b at once, as
+    plain fp64 matrix products over all heads: q_b [s_q, n_h, d_c + d_R],
+    S = rows . q^T, row r masked past position L - s_q + r, a = softmax(scale S)
+    per (r, head), u = a^T C.  Returns (u [s_q, n_h, d_c], lse [s_q, n_h]) and,
+    with want_abs, abs_c = a^T |C| [s_q, n_h, d_c] as a third value."""
+    rows = gather_rows(cache, block_table, w.page_size, b, L)
+    C = rows[:, :w.d_c]
+    absC = np.abs(C) if want_abs else None
+    s_q = q_b.shape[0]
+    u = np.empty((s_q, q_b.shape[1], w.d_c))
+    lse = np.empty((s_q, q_b.shape[1]))
+    abs_c = np.empty_like(u) if want_abs else None
+    for r in range(s_q):
+        n_valid = L - s_q + r + 1
+        S = w.softmax_scale * (rows[:n_valid] @ np.asarray(q_b[r], f64).T)   # [n_valid, n_h]
+        m = S.max(axis=0)
+        e = np.exp(S - m)
+        z = e.sum(axis=0)
+        a = e / z
+        u[r] = a.T @ C[:n_valid]
+        lse[r] = m + np.log(z)
+        if want_abs:
+            abs_c[r] = a.T @ absC[:n_valid]
+    return (u, lse, abs_c) if want_abs else (u, lse)
 
 
 def up_project(u: np.ndarray, W_UV: np.ndarray) -> np.ndarray:

@@ -82,9 +82,13 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.mla_absorb_weights(None, 16, 32, 128, 128, 512, 7168, 0, None) == INVALID
     assert lib.mla_absorb_weights(16, 32, 48, 0, 128, 512, 7168, 0, None) == INVALID
     assert lib.mla_absorb_weights(16, 32, 48, 128, 128, 512, 7168, 9, None) == INVALID
-    assert lib.mla_up_proj(16, 32, 48, 4, 0, 512, 128, 0, None) == INVALID
-    assert lib.mla_up_proj(None, 32, 48, 4, 128, 512, 128, 0, None) == INVALID
-    assert lib.mla_up_proj(16, 32, 48, 0, 128, 512, 128, 0, None) == OK      # T = 0: nothing to do
+    assert lib.mla_up_proj(16, 32, 48, 4, 0, 512, 128, 0, 0, None) == INVALID
+    assert lib.mla_up_proj(None, 32, 48, 4, 128, 512, 128, 0, 0, None) == INVALID
+    assert lib.mla_up_proj(16, 32, 48, 0, 128, 512, 128, 0, 0, None) == OK      # T = 0: nothing to do
+    assert lib.mla_up_proj(16, 32, 48, 4, 128, 512, 128, 0, 1, None) == INVALID  # bf16 u, fp32 W
+    assert lib.mla_up_proj(16, 32, 48, 4, 128, 512, 128, 3, 0, None) == INVALID  # u dtype
+    assert lib.mla_up_proj(16, 32, 48, 4, 128, 512, 129, 1, 0, None) == UNSUPPORTED  # d_v > 128
+    assert lib.mla_up_proj(16, 32, 48, 4, 128, 96, 128, 1, 0, None) == UNSUPPORTED   # bf16 d_c % 64
     assert lib.mla_form_query(16, 32, 48, 64, 80, 4, 128, 7168, 512, 63, 1e4, 0, None) == INVALID
     assert lib.mla_form_query(16, 32, 48, 64, 80, 4, 128, 7168, 512, 64, -1.0, 0, None) == INVALID
     assert lib.mla_form_query(16, 32, 48, 64, 80, 0, 128, 7168, 512, 64, 1e4, 0, None) == OK
@@ -101,6 +105,19 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError):
         mla._ptr(t)
     assert mla._ptr(None) is None
+
+
+def test_merge_binding_refuses_non_fp32_statistics():
+    # the merge kernel reads lse words as fp32; other dtypes are refused before
+    # any pointer is taken
+    import torch
+    u_parts = torch.zeros((2, 3, 8))
+    u = torch.zeros((3, 8))
+    for bad in (torch.float64, torch.bfloat16):
+        with pytest.raises(TypeError):
+            mla.mla_merge_partials(u_parts, torch.zeros((2, 3), dtype=bad), u)
+        with pytest.raises(TypeError):
+            mla.mla_merge_partials(u_parts, torch.zeros((2, 3)), u, torch.zeros(3, dtype=bad))
 
 
 @pytest.mark.parametrize("args,want", [

@@ -111,6 +111,34 @@ def test_absorbed_equals_expanded(use_wqk):
         assert abs(lse_a - lse) < 1e-10
 
 
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_all_heads_helpers_reproduce_the_expanded_definition(s_q):
+    # absorbed_queries + decode_absorbed_seq (all heads of a sequence as matrix
+    # products) must give the expanded oracle's o and lse through o = W^UV u
+    w = medium_workload(s_q=s_q)
+    inp = synth.draw(w)
+    ex = orc.decode_expanded(inp, w)
+    for b in range(w.B):
+        q_b = np.stack([orc.absorbed_queries(inp, w, b, r) for r in range(w.s_q)])
+        u, lse, abs_c = orc.decode_absorbed_seq(q_b, inp["cache"], inp["block_table"],
+                                                int(inp["seqlens"][b]), b, w, want_abs=True)
+        for r in range(w.s_q):
+            o = orc.up_project(u[r], inp["W_UV"])
+            for i in range(w.n_h):
+                o_ref, lse_ref = ex[(b, r, i)]
+                assert _max_abs(o[i], o_ref) < 1e-10
+                assert abs(lse[r, i] - lse_ref) < 1e-10
+        # the weighted absolute sum bounds |u| and is u itself when every
+        # latent is non-negative
+        assert np.all(abs_c >= np.abs(u) - 1e-12)
+    cache = np.abs(inp["cache"])
+    b = 0
+    q_b = np.stack([orc.absorbed_queries(inp, w, b, r) for r in range(w.s_q)])
+    u, _, abs_c = orc.decode_absorbed_seq(q_b, cache, inp["block_table"], int(inp["seqlens"][b]),
+                                          b, w, want_abs=True)
+    assert _max_abs(abs_c, u) < 1e-12
+
+
 def test_absorbed_scores_equal_expanded_scores():
     rng = np.random.default_rng(3)
     n_h, d_h, d_c, d_model = 3, 5, 7, 11

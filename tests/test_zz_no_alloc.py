@@ -4,16 +4,18 @@ Some callers (a host framework that owns all device memory, a plugin
 interface that passes no workspace) cannot give the library scratch space.
 For them mla_decode_noalloc uses a fixed array inside the library instead
 of a workspace.  This file checks, through the C ABI, that it returns what
-mla_decode returns, on two calls in a row with different inputs (the second
-call finds the first call's data still in the shared array), and that
-parameters needing more than the array's 32 MiB are refused up front.
+mla_decode returns bit for bit (both run the same kernels on the same
+chunking, so any difference would be stale data in the shared array), on
+two calls in a row with different inputs (the second call finds the first
+call's data still in the shared array), and that parameters needing more
+than the array's 32 MiB are refused up front.
 The file is named to run last.
 """
 import numpy as np
 import pytest
 import torch
 
-from gpu_pipeline import ATOL_REL, LSE_REL, f64, lse_err, to_dev, to_dev_i32
+from gpu_pipeline import to_dev, to_dev_i32
 from mla_latent_kv_23_b200 import mla, synth
 
 pytestmark = pytest.mark.gpu
@@ -42,10 +44,7 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
         mla.mla_decode_noalloc(p)
         torch.cuda.synchronize()
         assert mla.mla_check_device_errors() == 0
-        ur, uu = f64(u_ref), f64(u)
-        assert np.max(np.abs(uu - ur) / (1 + np.abs(ur))) <= ATOL_REL
-        lr, ll = f64(lse_ref), f64(lse)
-        assert max(lse_err(a, b) for a, b in zip(ll.ravel(), lr.ravel())) <= LSE_REL
+        assert torch.equal(u, u_ref) and torch.equal(lse, lse_ref)
 
 
 def test_noalloc_refuses_parameters_beyond_its_array():
