@@ -28,7 +28,8 @@ struct DeviceInfo {
   bool ready = false;
   int sm_count = 0;
   int cc_major = 0, cc_minor = 0;
-  int max_clusters = 0;  // co-resident 2-CTA clusters of the tensor-core kernel
+  int max_clusters = 0;  // co-resident 2-CTA clusters of the DeepSeek-V3-shape kernel
+  bool small_tc = false;  // the small-latent tensor-core kernel is usable
   bool up_proj_tc = false;
   int* flags = nullptr;  // device address of g_device_flags
 };
@@ -65,6 +66,7 @@ mla_status device_info(const DeviceInfo** out) {
     if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.flags), g_device_flags)) != cudaSuccess)
       return cuda_status(e);
     d.max_clusters = (d.cc_major == 10) ? decode_sm100_prepare() : 0;
+    d.small_tc = (d.cc_major == 10) && decode_small_sm100_prepare() != 0;
     d.up_proj_tc = (d.cc_major == 10) && up_proj_sm100_prepare() != 0;
     if (g_encode == nullptr) {
       cudaDriverEntryPointQueryResult q;
@@ -114,21 +116,29 @@ mla_status validate_decode(const mla_decode_params* p) {
   return MLA_OK;
 }
 
-bool use_tensor_cores(const mla_decode_params* p, const DeviceInfo* d) {
-  return d->cc_major == 10 && d->max_clusters > 0 && p->dtype == MLA_DTYPE_BF16 && p->d_c == 512 &&
-         p->d_R == 64 && g_encode != nullptr;
+// The attend kernels, each a tensor-core (tcgen05) kernel for its shapes:
+// the paired-CTA kernel for the DeepSeek-V3 shape (bf16, d_c = 512,
+// d_R = 64) and the one-CTA kernel for small latent widths.
+enum class Kernel { kNone, kV3, kSmall };
+
+Kernel select_kernel(const mla_decode_params* p, const DeviceInfo* d) {
+  if (d->cc_major != 10 || g_encode == nullptr) return Kernel::kNone;
+  const bool bf16 = p->dtype == MLA_DTYPE_BF16;
+  if (bf16 && p->d_c == 512 && p->d_R == 64 && d->max_clusters > 0) return Kernel::kV3;
+  if (d->small_tc && decode_small_sm100_supported(bf16, p->d_c, p->d_R)) return Kernel::kSmall;
+  return Kernel::kNone;
 }
 
 int choose_chunks(const mla_decode_params* p, const DeviceInfo* d) {
   if (p->num_splits > 0) return p->num_splits;
-  if (use_tensor_cores(p, d)) return std::max(1, d->max_clusters / p->s_q);
-  return std::max(1, (2 * d->sm_count) / (p->s_q * p->n_h));
+  if (select_kernel(p, d) == Kernel::kV3) return std::max(1, d->max_clusters / p->s_q);
+  return std::max(1, d->sm_count / p->s_q);  // one CTA per SM
 }
 
 struct Resolved {
   DecodeArgs a;
   long long slots = 0;  // partial rows per head the workspace holds
-  bool tc = false;
+  Kernel kernel = Kernel::kNone;
   const DeviceInfo* dev = nullptr;
 };
 
@@ -136,6 +146,8 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   mla_status st = validate_decode(p);
   if (st != MLA_OK) return st;
   if ((st = device_info(&r->dev)) != MLA_OK) return st;
+  r->kernel = select_kernel(p, r->dev);
+  if (r->kernel == Kernel::kNone) return MLA_ERR_UNSUPPORTED;
   const int G = choose_chunks(p, r->dev);
   if ((long long)G * p->s_q * 2 > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
   const WsLayout L = ws_layout(p->B, p->s_q, p->n_h, p->d_c, G);
@@ -170,8 +182,7 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   a.scale = p->softmax_scale;
   a.bf16 = p->dtype == MLA_DTYPE_BF16;
   a.out_f32 = p->u_fp32 != 0 || p->dtype == MLA_DTYPE_FP32;
-  r->tc = use_tensor_cores(p, r->dev);
-  a.part_bf16 = r->tc && !a.out_f32;
+  a.part_bf16 = r->kernel == Kernel::kV3 && !a.out_f32;
   a.pdl = false;
   return MLA_OK;
 }
@@ -222,7 +233,41 @@ mla_status encode_out(CUtensorMap* m, void* ptr, uint64_t n_h, uint64_t rows, bo
 // while the previous stage finishes.
 mla_status attend(Resolved r, const mla_decode_params* p, cudaStream_t s, bool pdl) {
   r.a.pdl = pdl;
-  if (!r.tc) return cuda_status(launch_decode_simt(r.a, s));
+  if (r.kernel == Kernel::kSmall) {
+    const bool f32 = !r.a.bf16;
+    const uint64_t es = f32 ? 4 : 2, W = (uint64_t)p->d_c + p->d_R;
+    const CUtensorMapDataType tdt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint32_t cols = static_cast<cuuint32_t>(128 / es);
+    CUtensorMap q_map, kv_map, kv_pv_map;
+    memset(&kv_pv_map, 0, sizeof(kv_pv_map));
+    {
+      const cuuint64_t dims[3] = {W, (cuuint64_t)p->n_h, (cuuint64_t)p->B * p->s_q};
+      const cuuint64_t strides[2] = {W * es, (cuuint64_t)p->n_h * W * es};
+      const cuuint32_t box[3] = {cols, 128, 1};
+      const cuuint32_t estr[3] = {1, 1, 1};
+      if (g_encode(&q_map, tdt, 3, const_cast<void*>(p->q), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    }
+    {
+      const cuuint64_t dims[2] = {W, (cuuint64_t)p->num_pages * p->page_size};
+      const cuuint64_t strides[1] = {W * es};
+      const cuuint32_t box[2] = {cols, (cuuint32_t)kTileTokens};
+      const cuuint32_t estr[2] = {1, 1};
+      if (g_encode(&kv_map, tdt, 2, const_cast<void*>(p->kv_cache), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+      // an MN-major tf32 operand: 128-byte swizzle of 32-byte atoms
+      if (f32 && g_encode(&kv_pv_map, tdt, 2, const_cast<void*>(p->kv_cache), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MLA_ERR_CUDA;
+    }
+    return cuda_status(launch_decode_small_sm100(r.a, q_map, kv_map, kv_pv_map, s));
+  }
   Sm100Maps maps;
   const uint64_t kvrows = (uint64_t)p->num_pages * p->page_size;
   mla_status st;
@@ -302,7 +347,7 @@ mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_c
   if (st != MLA_OK) return st;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != MLA_OK) return st;
-  if (uses_tensor_cores) *uses_tensor_cores = use_tensor_cores(p, d) ? 1 : 0;
+  if (uses_tensor_cores) *uses_tensor_cores = select_kernel(p, d) != Kernel::kNone ? 1 : 0;
   if (num_chunks) *num_chunks = choose_chunks(p, d);
   return MLA_OK;
 }

@@ -90,8 +90,8 @@ constexpr uint32_t kPHalf = 64 * 64;                     // 64 heads x 32 tokens
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKv = kOffQ + kQBytes;
 constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;   // [2] second halves of P
-constexpr uint32_t kOffRed = kOffP + 2 * kPHalf;             // float [2 parity][2 c][64 heads]
-constexpr uint32_t kOffSum = kOffRed + 2 * 2 * 64 * 4;       // float [2 kind][2 c][64 heads]
+constexpr uint32_t kOffMax = kOffP + 2 * kPHalf;             // float [2 tile parity][64 heads]
+constexpr uint32_t kOffSum = kOffMax + 2 * 64 * 4;           // float [2 kind][2 group][64 heads]
 constexpr uint32_t kOffScratch = kOffSum + 2 * 2 * 64 * 4;    // 16 words written by the odd CTA's signals
 constexpr uint32_t kOffBar = kOffScratch + 64;
 
@@ -110,7 +110,8 @@ enum Bar {
   Q_LOCAL = PV_DONE + 2,           // this CTA's query bytes
   Q_FULL,                          // even CTA, paired: both queries in place (relays)
   Q_EMPTY,                         // last S of a segment done (paired commit)
-  GRP,                             // the 8 softmax warps of this CTA
+  DEC,                             // [2] per softmax group: its 4 warps decided a tile's maximum
+  GRP = DEC + 2,                   // the 8 softmax warps of this CTA
   EPI_FREE,                        // the 8 softmax warps' output stores have read the query area
   MMA_FINAL,                       // even CTA: all S issued so far are complete
   MMA_FINAL_PV,                    // even CTA: all P . C issued so far are complete
@@ -219,8 +220,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(S_FULL + i), 1);
-      mbar_init(bar(S_EMPTY + i), 8);
-      mbar_init(bar(P_FULL + i), 8);
+      mbar_init(bar(S_EMPTY + i), 4);
+      mbar_init(bar(P_FULL + i), 4);
+      mbar_init(bar(DEC + i), 4);
       mbar_init(bar(PV_DONE + i), 1);
     }
     mbar_init(bar(Q_LOCAL), 1);
@@ -503,22 +505,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpSoftmax0) {
     // ------------------------------------------------------------ softmax
+    // Two groups of four warps take alternate tiles (group = g & 1, which is
+    // also the tile's S buffer and P ring slot); warp q of a group reads TMEM
+    // lanes [32q, 32q + 32) for all 64 tokens, so a head's tile maximum needs
+    // no exchange between warps.  The running maximum after tile g is
+    // published per head in shared memory (slot g & 1); a group decides tile
+    // g from the maximum after tile g - 1, which the other group published.
     const int sw_warp = warp - kWarpSoftmax0;       // 0..7
-    const int c = sw_warp >> 2;                     // tokens [32c, 32c + 32) of a tile
+    const int grp = sw_warp >> 2;                   // softmax group; also the O block it drains
+    const int gw = sw_warp & 3;                     // warp within the group
     const int qd = warp & 3;                        // TMEM lanes [32 qd, 32 qd + 32)
     const int jh = lane >> 4;                       // S row half: partial over CTA jh's columns
     const int hS = 16 * qd + (lane & 15);           // head (local) of this thread's S row
     const int hO = (32 * qd + lane) & 63;           // head (local) of this thread's O lane
     const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     const uint32_t sw64 = static_cast<uint32_t>((hS >> 1) & 3);  // 64-byte swizzle of row hS
-    float* red = reinterpret_cast<float*>(base + kOffRed);   // [parity][c][head]
-    float* sums = reinterpret_cast<float*>(base + kOffSum);  // [kind][c][head]
+    float* mx_pub = reinterpret_cast<float*>(base + kOffMax);  // [tile parity][head]
+    float* sums = reinterpret_cast<float*>(base + kOffSum);    // [kind][group][head]
     const float c_log2 = p.scale_log2;
     uint32_t grp_phase = 0;
-    auto rendezvous = [&]() -> bool {
+    // A failed wait (a broken protocol) sets the device flag; the warp then
+    // skips its later waits but still runs every step, so that the group's
+    // named barriers and the other roles' waits stay matched and the kernel
+    // ends.
+    auto rendezvous = [&](bool live) -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(GRP));
-      return warp_wait(bar(GRP), (grp_phase++) & 1, p.err);
+      const uint32_t ph = (grp_phase++) & 1;
+      return live && warp_wait(bar(GRP), ph, p.err);
     };
 
     ChunkWalk walk;
@@ -526,85 +540,103 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Segment sg;
     int g = 0;
     bool ok = true;
-    while (ok && walk.next(sg)) {
+    while (walk.next(sg)) {
       const int L = p.seqlens[sg.b];
       const int L_eff = L - p.s_q + 1 + qrow;  // positions this query row may see
       const int n_t = sg.t1 - sg.t0;
+      const int g0 = g;
       // the segment's output row: u's row, or its partial slot (read now,
       // used by the epilogue)
       const int out_z =
           sg.whole ? sg.b * p.s_q + qrow : (p.split_base[sg.b] + sg.part) * p.s_q + qrow;
-      // m_s: running max of the S head (weights); m_o: the same sequence of
-      // values for the O head (rescaling), derived from the same shared maxima
-      float m_s = -INFINITY, m_o = -INFINITY, l = 0.f, l_exact = 0.f;
-      for (int jt = 0; jt < n_t; ++jt, ++g) {
+      // this group's sums over its own tiles of the segment, in the scale of
+      // m_used (the maximum it last applied)
+      float m_used = -INFINITY, l = 0.f, l_exact = 0.f;
+      for (int jt = (grp - g0) & 1; jt < n_t; jt += 2) {
+        const int gt = g0 + jt;
         const int t = sg.t0 + jt;
-        // ---- partial scores of tile g -> registers; free the S buffer
-        if (!(ok = warp_wait(bar(S_FULL + (g & 1)), (g >> 1) & 1, p.err))) break;
+        // ---- partial scores of tile gt -> registers; free the S buffer
+        ok = ok && warp_wait(bar(S_FULL + grp), (gt >> 1) & 1, p.err);
         tc_fence_after();
-        float own[32];
-        {
+        // sc[16 c + k]: token 32 c + 16 jh + k of the tile, for head hS.
+        // S = partial(CTA 0 columns) + partial(CTA 1 columns): lane jh keeps
+        // tokens [16 jh, 16 jh + 16) of each 32 and hands the rest to lane ^ 16
+        float sc[32];
+        const uint32_t sb = tmem + lane_base + kTmemS + grp * 128;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           float va[32], vb[32];
-          const uint32_t sb = tmem + lane_base + kTmemS + (g & 1) * 128 + 32 * c;
-          tmem_ld32(sb, va);
-          tmem_ld32(sb + 64, vb);
+          tmem_ld32(sb + 32 * c, va);
+          tmem_ld32(sb + 64 + 32 * c, vb);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) own[k] = jh ? vb[k] : va[k];
+          for (int k = 0; k < 16; ++k) {
+            const float own_lo = jh ? vb[k] : va[k], own_hi = jh ? vb[16 + k] : va[16 + k];
+            const float send = jh ? own_lo : own_hi;
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            sc[16 * c + k] = (jh ? own_hi : own_lo) + recv;
+          }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) signal_lead(S_EMPTY + (g & 1), sw_warp == 0, 32u, sw_warp);
-        // S = partial(CTA 0 columns) + partial(CTA 1 columns): lane jh keeps
-        // tokens [16 jh, 16 jh + 16) of its 32 and hands the rest to lane ^ 16
-        float sc[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float send = jh ? own[k] : own[16 + k];
-          const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-          sc[k] = (jh ? own[16 + k] : own[k]) + recv;
-        }
-        const int nv = L_eff - (t * kTileTokens + 32 * c + 16 * jh);  // valid of these 16
-        if (nv < 16) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            if (k >= nv) sc[k] = -INFINITY;
-        }
+        if (lane == 0) signal_lead(S_EMPTY + grp, gw == 0, 16u, gw);
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 16; k += 2) {
-          mx0 = fmaxf(mx0, sc[k]);
-          mx1 = fmaxf(mx1, sc[k + 1]);
+        for (int c = 0; c < 2; ++c) {
+          const int nv = L_eff - (t * kTileTokens + 32 * c + 16 * jh);  // valid of these 16
+          if (nv < 16) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              if (k >= nv) sc[16 * c + k] = -INFINITY;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; k += 2) {
+            mx0 = fmaxf(mx0, sc[16 * c + k]);
+            mx1 = fmaxf(mx1, sc[16 * c + k + 1]);
+          }
         }
         float mx = fmaxf(mx0, mx1);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        if (jh == 0) red[((g & 1) * 2 + c) * 64 + hS] = mx;
-        if (!(ok = rendezvous())) break;
-        // tile maximum (raw scores; scale > 0 commutes with max), the same
-        // expression for the S head and for the O head
-        const float* rd = red + (g & 1) * 2 * 64;
-        const float t_s = fmaxf(rd[hS], rd[64 + hS]) * c_log2;
-        const float t_o = fmaxf(rd[hO], rd[64 + hO]) * c_log2;
-        float alpha_s = 1.f, alpha_o = 1.f;
+        // ---- the maximum after this tile.  The running maximum may go
+        // stale: it moves only when a tile's maximum exceeds it by more than
+        // 2^kRescaleThreshold (weights stay below that factor), which keeps O
+        // rescales rare.  Raw scores: scale > 0 commutes with max.
+        const float t_s = mx * c_log2;
+        float m_prev = -INFINITY;
+        if (jt > 0) {  // tile gt - 1 (the other group's) is in this segment
+          ok = ok && warp_wait(bar(DEC + (grp ^ 1)), ((gt - 1) >> 1) & 1, p.err);
+          m_prev = mx_pub[((gt - 1) & 1) * 64 + hS];
+        }
+        const float m_new = (m_prev == -INFINITY || t_s > m_prev + kRescaleThreshold)
+                                ? fmaxf(m_prev, t_s) : m_prev;
+        if (jh == 0) mx_pub[(gt & 1) * 64 + hS] = m_new;
+        named_bar_sync(1 + grp, 128);
+        // O lane hO: rescale if its head's maximum moved at this tile
+        float alpha_o = 1.f;
         bool resc_o = false;
-        {
-          const float mn = fmaxf(m_s, t_s);
-          if (mn > m_s + kRescaleThreshold) {
-            alpha_s = ex2_approx(m_s - mn);
-            m_s = mn;
-          }
-          const float mo = fmaxf(m_o, t_o);
-          if (mo > m_o + kRescaleThreshold) {
-            alpha_o = ex2_approx(m_o - mo);
-            m_o = mo;
+        if (jt > 0) {
+          const float mo_prev = mx_pub[((gt - 1) & 1) * 64 + hO];
+          const float mo_new = mx_pub[(gt & 1) * 64 + hO];
+          if (mo_new != mo_prev) {
+            alpha_o = ex2_approx(mo_prev - mo_new);  // mo_prev = -inf: O holds only zeros
             resc_o = true;
           }
         }
-        const float neg_m = m_s == -INFINITY ? 0.f : -m_s;
+        // the decision of tile gt is published (and slot (gt - 1) & 1 read)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(DEC + grp));
+        // this group's sums move to the new scale
+        if (m_new != m_used) {
+          const float f = m_used == -INFINITY ? 0.f : ex2_approx(m_used - m_new);
+          l *= f;
+          l_exact *= f;
+          m_used = m_new;
+        }
+        const float neg_m = m_new == -INFINITY ? 0.f : -m_new;
         float r0 = 0.f, r1 = 0.f, e0 = 0.f, e1 = 0.f;
-        uint32_t pk[8];
+        uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 16; k += 2) {
+        for (int k = 0; k < 32; k += 2) {
           const float a = ex2_approx(fmaf(sc[k], c_log2, neg_m));
           const float b = ex2_approx(fmaf(sc[k + 1], c_log2, neg_m));
           const __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
@@ -614,64 +646,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         // u is normalised by the sum of the rounded weights it was built
         // from; lse uses the unrounded weights
-        l = l * alpha_s + (r0 + r1);
-        l_exact = l_exact * alpha_s + (e0 + e1);
+        l += r0 + r1;
+        l_exact += e0 + e1;
 
-        // P's second-half slot g&1 was last read by PV_{g-2}; O may be
-        // rescaled only after PV_{g-1} (tiles of an earlier segment were
-        // retired by that segment's epilogue, and the first P . C of a segment
+        // P's ring slot grp was last read by PV(gt - 2); O may be rescaled
+        // only after PV(gt - 1) (tiles of an earlier segment were retired by
+        // that segment's epilogue, and the first P . C of a segment
         // overwrites O)
-        if (jt >= 2 && !(ok = warp_wait(bar(PV_DONE + (g & 1)), ((g - 2) >> 1) & 1, p.err)))
-          break;
-        if (jt >= 1 && __any_sync(0xffffffffu, resc_o)) {
-          if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err)))
-            break;
+        if (gt >= 2) ok = ok && warp_wait(bar(PV_DONE + grp), ((gt - 2) >> 1) & 1, p.err);
+        if (__any_sync(0xffffffffu, resc_o)) {
+          ok = ok && warp_wait(bar(PV_DONE + (grp ^ 1)), ((gt - 1) >> 1) & 1, p.err);
           tc_fence_after();
-          for (int c0 = 0; c0 < 128; c0 += 32) {
+          for (int c0 = 0; c0 < 256; c0 += 32) {  // both O blocks of these lanes
             float o[32];
-            tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
+            tmem_ld32(tmem + lane_base + kTmemO + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha_o;
-            tmem_st32(tmem + lane_base + kTmemO + c * 128 + c0, o);
+            tmem_st32(tmem + lane_base + kTmemO + c0, o);
           }
           tmem_wait_st();
         }
         // P row hS, tokens [32c + 16jh, +16): half c of the row (32 tokens =
         // 64 B, 64-byte swizzle) lives in the stage's RoPE block (c = 0) or
-        // in second-half slot g&1 (c = 1); 16-byte chunks 2jh and 2jh + 1
-        const uint32_t prow =
-            (c == 0 ? sbase + kOffKv + (g % kStages) * kStageBytes + 4 * kKvBlk
-                    : sbase + kOffP + (g & 1) * kPHalf) + hS * 64;
+        // in ring slot grp (c = 1); 16-byte chunks 2jh and 2jh + 1
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const uint32_t ch = static_cast<uint32_t>(2 * jh + k);
-          st_shared_v4(prow + ((ch ^ sw64) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
-                       pk[4 * k + 3]);
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t prow =
+              (c == 0 ? sbase + kOffKv + (gt % kStages) * kStageBytes + 4 * kKvBlk
+                      : sbase + kOffP + grp * kPHalf) + hS * 64;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const uint32_t ch = static_cast<uint32_t>(2 * jh + k);
+            st_shared_v4(prow + ((ch ^ sw64) << 4), pk[8 * c + 4 * k], pk[8 * c + 4 * k + 1],
+                         pk[8 * c + 4 * k + 2], pk[8 * c + 4 * k + 3]);
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) signal_lead(P_FULL + (g & 1), sw_warp == 0, 32u, sw_warp);
+        if (lane == 0) signal_lead(P_FULL + grp, gw == 0, 16u, gw);
       }
-      if (!ok) break;
+      g = g0 + n_t;
 
       // ---- epilogue: u = O / l for this thread's O lane (one head, 128
-      // consecutive latent columns)
+      // consecutive latent columns of O block grp)
+      // the maximum after the segment's last tile (decided by either group)
+      if (((g - 1) & 1) != grp) ok = ok && warp_wait(bar(DEC + (grp ^ 1)), ((g - 1) >> 1) & 1, p.err);
+      const float mS_fin = mx_pub[((g - 1) & 1) * 64 + hS];
+      const float mO_fin = mx_pub[((g - 1) & 1) * 64 + hO];
       {
-        const float l2 = l + __shfl_xor_sync(0xffffffffu, l, 16);
-        const float e2 = l_exact + __shfl_xor_sync(0xffffffffu, l_exact, 16);
+        // this group's sums in the scale of the final maximum
+        const float f = m_used == mS_fin ? 1.f : m_used == -INFINITY ? 0.f : ex2_approx(m_used - mS_fin);
+        const float lf = l * f, lef = l_exact * f;
+        const float l2 = lf + __shfl_xor_sync(0xffffffffu, lf, 16);
+        const float e2 = lef + __shfl_xor_sync(0xffffffffu, lef, 16);
         if (jh == 0) {
-          sums[(0 * 2 + c) * 64 + hS] = l2;
-          sums[(1 * 2 + c) * 64 + hS] = e2;
+          sums[(0 * 2 + grp) * 64 + hS] = l2;
+          sums[(1 * 2 + grp) * 64 + hS] = e2;
         }
       }
-      if (!(ok = rendezvous())) break;
+      // every warp has read the published maxima of this segment before any
+      // starts the next one
+      ok = rendezvous(ok);
       const float l_o = sums[(0 * 2 + 0) * 64 + hO] + sums[(0 * 2 + 1) * 64 + hO];
       const float le_o = sums[(1 * 2 + 0) * 64 + hO] + sums[(1 * 2 + 1) * 64 + hO];
-      if (!(ok = warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err))) break;
+      ok = ok && warp_wait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, p.err);
       tc_fence_after();
       const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
+      const int c = grp;                          // O block drained by this group
       const int col0 = 256 * c + 128 * (qd >> 1);  // latent column of TMEM column kTmemO + 128c
       // The segment's last S has read Q, so the query area stages the output:
       // 8 KB per warp, its 32 heads x 128 columns as boxes of 128-byte lines
@@ -741,7 +784,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const int head = 64 * (int)rank + hO;
       if (head < p.n_h && qd < 2 && c == 0) {
-        const float lse = le_o > 0.f ? (m_o + log2f(le_o)) * 0.69314718055994531f : -INFINITY;
+        const float lse = le_o > 0.f ? (mO_fin + log2f(le_o)) * 0.69314718055994531f : -INFINITY;
         if (sg.whole) {
           if (p.lse != nullptr) p.lse[(size_t)out_z * p.n_h + head] = lse;
         } else {

@@ -57,7 +57,19 @@ struct DecodeArgs {
 
 cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
-cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s);
+
+// Tensor-core decode for small latent widths (one CTA per KV chunk and query
+// row): fp32 with d_c a multiple of 32, d_c + d_R <= 128 (tf32), or bf16 with
+// d_c a multiple of 64, d_c + d_R <= 256.  q_map: q [B * s_q, n_h, d_c + d_R]
+// with boxes of 128 bytes x 128 heads x 1; kv_map: the cache [rows, d_c + d_R]
+// with boxes of 128 bytes x 64 rows; both 128-byte swizzle.  kv_pv_map (fp32
+// only): the cache again with 128-byte swizzle of 32-byte atoms.  Split
+// partials are fp32.
+bool decode_small_sm100_supported(bool bf16, int d_c, int d_R);
+int decode_small_sm100_prepare();
+cudaError_t launch_decode_small_sm100(const DecodeArgs& a, const CUtensorMap& q_map,
+                                      const CUtensorMap& kv_map, const CUtensorMap& kv_pv_map,
+                                      cudaStream_t s);
 
 // Tensor-core decode for n_h <= 128, d_c = 512, d_R = 64, bf16.
 // kv maps over the cache [rows, 576]: latent boxes 64 x 64 rows (128-byte

@@ -449,6 +449,10 @@ __device__ __forceinline__ void pdl_wait_previous() {
 // 61-63 (2 = 128-byte swizzle, 4 = 64-byte swizzle).
 constexpr uint32_t kLayoutSW128 = 2;
 constexpr uint32_t kLayoutSW64 = 4;
+// 128-byte swizzle of 32-byte atoms: the layout an MN-major operand of
+// 32-bit elements (tf32) must have; TMA writes it with
+// CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.
+constexpr uint32_t kLayoutSW128Atom32 = 1;
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
                                               uint32_t layout) {
   uint64_t d = 0;

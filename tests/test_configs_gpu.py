@@ -93,9 +93,15 @@ def test_long_context_stress():
 
 
 def test_tiny_config_all_outputs():
+    # fp32 throughout: the decode runs on the small-latent tensor-core kernel
+    # (tf32) and the up-projection as tf32 MMAs
     w = synth.config("tiny")
     inp = synth.draw(w)
     out = run_pipeline(w, inp)
+    p = mla.decode_params(out["q"], out["cache"], out["bt"], out["seqlens"], out["u"], out["lse"],
+                          w.page_size, w.d_R, w.softmax_scale)
+    tc, _ = mla.mla_decode_kernel_info(p)
+    assert tc == 1
     res = check_expanded(w, inp, out)
     assert res["n"] == w.B * w.s_q * w.n_h
     assert_parity(res)

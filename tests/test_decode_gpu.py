@@ -91,14 +91,50 @@ def test_garbage_past_sequence_end_is_ignored():
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_cuda_core_path_small_latent(dtype):
-    # d_c = 64, d_R = 16 goes to the CUDA-core kernel in either dtype
-    w = synth.config("tiny").with_(dtype=dtype, B=3, seqlens=(129, 129, 129), page_size=192,
-                                   block_table="permuted", full_pipeline=False)
+@pytest.mark.parametrize("s_q,splits", [(1, 4), (1, 0), (2, 3)])
+def test_small_latent_tensor_core_path(dtype, s_q, splits):
+    # d_c = 64, d_R = 16 runs on the small-latent tcgen05 kernel: tf32 for
+    # fp32 tensors, bf16 otherwise; a permuted block table, pages of 192
+    # tokens, a ragged tail (129 = 2 tiles + 1) and split rows
+    w = synth.config("tiny").with_(dtype=dtype, B=3, s_q=s_q, seqlens=(129, 129, 129),
+                                   page_size=192, block_table="permuted", full_pipeline=False)
     inp = synth.draw(w)
-    out = run_pipeline(w, inp, num_splits=4)
+    out = run_pipeline(w, inp, num_splits=splits)
+    p = mla.decode_params(out["q"], out["cache"], out["bt"], out["seqlens"], out["u"], out["lse"],
+                          w.page_size, w.d_R, w.softmax_scale, splits)
+    tc, _ = mla.mla_decode_kernel_info(p)
+    assert tc == 1
     res = check_expanded(w, inp, out)
+    assert res["n"] == w.B * w.s_q * w.n_h
     assert_parity(res)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_small_latent_on_exact_inputs(dtype):
+    # the same q on both sides, many tiles and chunks, s_q = 2 with lengths
+    # that leave a query row's last tile empty (65 = 64 + 1)
+    w = synth.Workload(name="small-exact", B=4, s_q=2, n_h=8, d_model=64, d_c=64, d_h=32,
+                       d_v=32, d_R=16, page_size=64, dtype=dtype, seqlens=(65, 700, 2, 1000),
+                       block_table="permuted", seed=9)
+    inp = synth.draw(w)
+    q = synth.random_q(w)
+    out = run_pipeline(w, inp, num_splits=7, q=to_dev(q, w))
+    picks = [(b, r, i) for b in range(w.B) for r in range(w.s_q) for i in range(w.n_h)]
+    res = check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"])
+    assert_parity(res)
+    if dtype == "bf16":
+        assert_tight(res)
+
+
+def test_unsupported_latent_widths_are_refused():
+    # no attend kernel for these shapes: refused before anything runs
+    q = torch.zeros((1, 1, 8, 96 + 16), dtype=torch.bfloat16, device="cuda")
+    cache = torch.zeros((64, 96 + 16), dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    sl = torch.ones((1,), dtype=torch.int32, device="cuda")
+    with pytest.raises(mla.MLAError) as e:
+        mla.decode(q, cache, bt, sl, 64, 16, 0.1)
+    assert e.value.status == 2   # MLA_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("u_dtype", [torch.float32, torch.bfloat16])
