@@ -132,4 +132,34 @@ cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_
 cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, void* o, int* err,
                                       int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s);
 
+// Weight-streaming projection Y[m, t] = sum_k W[m, k] X[t, k] on the tensor
+// cores (bf16): one CTA per (128-row tile, K slice), fp32 split-K
+// reduction in a workspace that is zero on entry and left zero.  w_map[0]
+// covers tiles [0, tiles0), w_map[1] the rest (boxes 64 x 128 rows); x_map:
+// X [N, K], box 64 x n_pad rows; all 128-byte swizzle, K a multiple of 64.
+// mode 0: query (W^Q rows -> q^nope -> W^UK^T on the tensor cores into
+// q[t, i, 0:d_c]; W^QR rows -> RoPE into q[t, i, d_c:]); mode 1: cache rows
+// [W^DKV h || RoPE(W^KR h)] through the block table; mode 2: y[t, m]
+// (pair = 2: X rows 2t, 2t + 1 are two terms of token t and are added).
+struct WgemmLaunch {
+  CUtensorMap w_map[2];
+  CUtensorMap x_map;
+  CUtensorMap uk_map;  // mode 0: W^UK as [n_h * 128, d_c], box 64 x 128 rows
+  int tiles, tiles0;
+  int K, N, n_pad, ksplit;
+  void* workspace;
+  int* err;
+  int mode;
+  void* out;
+  int n_h, d_c, d_R, ldo, pair;
+  const int* pos;
+  const int* seq;
+  const int* block_table;
+  int max_pages, page_size, num_pages;
+  float rope_base;
+};
+int wgemm_sm100_prepare();
+size_t wgemm_workspace_bytes(int tiles, int n_pad);
+cudaError_t launch_wgemm(const WgemmLaunch& L, cudaStream_t s);
+
 }  // namespace mla
