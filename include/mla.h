@@ -75,6 +75,23 @@ mla_status mla_absorb_weights(const void* W_UK, const void* W_Q, void* W_QK, int
                               int d_c, int d_model, mla_dtype dtype, void* stream);
 
 /*
+ * Projections around the attention (query formation, latent append, output
+ * projection) stream their weights once through the tensor cores; their K
+ * dimension is split over CTAs whose partial sums meet in an fp32 scratch
+ * area.  `workspace` (bf16 calls) is caller-owned device memory of at least
+ * mla_projection_workspace_size bytes, 256-byte aligned, that must be ZERO
+ * before its first use; every call leaves it zero again, so one zeroed
+ * workspace serves any number of calls ordered on one stream.  rows0 and
+ * rows1 are the row counts of the call's first and second weight tensor
+ * (n_h * d_c and n_h * d_R for mla_form_query, n_h * d_h and n_h * d_R for
+ * mla_form_query_fused, d_c and d_R for mla_append_latent, M and 0 for
+ * mla_output_projection); x_fp32_K is K for mla_output_projection with an
+ * fp32 x, else 0.
+ */
+mla_status mla_projection_workspace_size(int rows0, int rows1, int T, int x_fp32_K,
+                                         size_t* bytes);
+
+/*
  * Absorbed query formation ("MLA deep compression", absorption section score
  * equation and decoupled-RoPE section):
  *   q[t, i, 0:d_c]       = W_QK[i] . h[t]
@@ -86,10 +103,38 @@ mla_status mla_absorb_weights(const void* W_UK, const void* W_Q, void* W_QK, int
  *   W_QR  [n_h, d_R, d_model]      device, read
  *   pos   [T] int32                device, read (query positions)
  *   q     [T, n_h, d_c + d_R]      device, written (T = B * s_q rows)
+ * bf16: tensor cores (d_model a multiple of 64, d_R dividing 128), with a
+ * projection workspace; fp32: a tiled CUDA-core GEMM (workspace unused).
  */
 mla_status mla_form_query(const void* h, const void* W_QK, const void* W_QR, const int* pos,
                           void* q, int T, int n_h, int d_model, int d_c, int d_R, float rope_base,
-                          mla_dtype dtype, void* stream);
+                          mla_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Query formation with the absorption done on the fly ("MLA deep
+ * compression", absorption section, score equation read right to left, and
+ * decoupled-RoPE section): no precomputed W_QK is read.
+ *   q[t, i, 0:d_c]       = W_UK[i]^T . (W_Q[i] . h[t])
+ *   q[t, i, d_c:d_c+d_R] = RoPE(W_QR[i] . h[t], pos[t])
+ * bf16, one kernel: the products with W_Q and W_QR stream those weights once
+ * through the tensor cores; the CTA that completes head i's W_Q . h applies
+ * W_UK[i]^T on the tensor cores (W_Q . h split into two bf16 terms, so it
+ * enters unrounded).  Reads 2 * n_h * (d_h + d_R) * d_model + 2 * n_h * d_h
+ * * d_c bytes of weights (369 MB at the DeepSeek-V3 shape) instead of the
+ * absorbed path's 2 * n_h * (d_c + d_R) * d_model (1057 MB).
+ *   h     [T, d_model]        device, read (bf16)
+ *   W_Q   [n_h, d_h, d_model] device, read
+ *   W_UK  [n_h, d_h, d_c]     device, read
+ *   W_QR  [n_h, d_R, d_model] device, read
+ *   pos   [T] int32           device, read
+ *   q     [T, n_h, d_c + d_R] device, written
+ * Supported: d_h = 128, d_c a multiple of 128 up to 512, d_model a multiple
+ * of 64, d_R even and dividing 128.  Needs a projection workspace.
+ */
+mla_status mla_form_query_fused(const void* h, const void* W_Q, const void* W_UK,
+                                const void* W_QR, const int* pos, void* q, int T, int n_h,
+                                int d_h, int d_model, int d_c, int d_R, float rope_base,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Latent append ("MLA deep compression", low-rank projection section and
@@ -104,12 +149,15 @@ mla_status mla_form_query(const void* h, const void* W_QK, const void* W_QR, con
  *   block_table [*, max_pages_per_seq] int32      device, read
  *   kv_cache    [num_pages*page_size, d_c + d_R]  device, written (only the T rows)
  * Out-of-range page ids raise MLA_DEVFLAG_BAD_PAGE and the row is skipped.
+ * bf16: tensor cores (d_model a multiple of 64, d_R <= 128), with a
+ * projection workspace; fp32: a tiled CUDA-core GEMM (workspace unused).
  */
 mla_status mla_append_latent(const void* h, const void* W_DKV, const void* W_KR,
                              const int* seq_ids, const int* pos, const int* block_table,
                              int max_pages_per_seq, int page_size, int num_pages, void* kv_cache,
                              int T, int d_model, int d_c, int d_R, float rope_base,
-                             mla_dtype dtype, void* stream);
+                             mla_dtype dtype, void* workspace, size_t workspace_bytes,
+                             void* stream);
 
 /*
  * Absorbed decode over a paged latent cache ("MLA deep compression",
@@ -220,6 +268,35 @@ mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_c
  */
 mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h, int d_c,
                        int d_v, mla_dtype u_dtype, mla_dtype dtype, void* stream);
+
+/*
+ * Output side folded offline ("Attention-head anatomy" section 5: W^UV folds
+ * into W^O; "MLA deep compression", absorption section, output equation):
+ *   W_OUV[m, i * d_c + c] = sum_v W_O[m, i * d_v + v] W_UV[i, v, c]
+ * so that y = W_O . concat_i(W_UV[i] u_i) = W_OUV . concat_i(u_i).
+ *   W_O    [d_model, n_h * d_v]   device, read
+ *   W_UV   [n_h, d_v, d_c]        device, read
+ *   W_OUV  [d_model, n_h * d_c]   device, written
+ * Run once per model (tiled CUDA-core GEMM, fp32 accumulation).
+ */
+mla_status mla_fold_output_weights(const void* W_O, const void* W_UV, void* W_OUV, int n_h, int d_v,
+                                   int d_c, int d_model, mla_dtype dtype, void* stream);
+
+/*
+ * Output projection y[t, m] = sum_k W[m, k] x[t, k] on the tensor cores,
+ * streaming W once: with W = W_OUV and x = u flattened [T, n_h * d_c] it
+ * projects the decode's u straight to the hidden size; with W = W_O and
+ * x = o flattened [T, n_h * d_v] it is the unfolded output projection.
+ *   x  [T, K]  device, read; bf16, or fp32 (split into two bf16 terms whose
+ *              products are added, so x enters to within 2^-16 of itself)
+ *   W  [M, K]  device, read, bf16
+ *   y  [T, M]  device, written, bf16
+ * K a multiple of 64, M a multiple of 8.  Needs a projection workspace
+ * (rows0 = M, rows1 = 0, x_fp32_K = K for an fp32 x).
+ */
+mla_status mla_output_projection(const void* x, mla_dtype x_dtype, const void* W, void* y, int T,
+                                 int K, int M, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /*
  * Merge of partial decode results over disjoint parts of the same query

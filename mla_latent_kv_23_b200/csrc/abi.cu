@@ -8,6 +8,7 @@
 #include <climits>
 #include <cmath>
 #include <cstring>
+#include <functional>
 #include <mutex>
 
 #include "internal.h"
@@ -31,6 +32,7 @@ struct DeviceInfo {
   int max_clusters = 0;  // co-resident 2-CTA clusters of the DeepSeek-V3-shape kernel
   bool small_tc = false;  // the small-latent tensor-core kernel is usable
   bool up_proj_tc = false;
+  bool wgemm_tc = false;  // the weight-streaming projection kernel is usable
   int* flags = nullptr;  // device address of g_device_flags
 };
 
@@ -68,6 +70,7 @@ mla_status device_info(const DeviceInfo** out) {
     d.max_clusters = (d.cc_major == 10) ? decode_sm100_prepare() : 0;
     d.small_tc = (d.cc_major == 10) && decode_small_sm100_prepare() != 0;
     d.up_proj_tc = (d.cc_major == 10) && up_proj_sm100_prepare() != 0;
+    d.wgemm_tc = (d.cc_major == 10) && wgemm_sm100_prepare() != 0;
     if (g_encode == nullptr) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -197,6 +200,47 @@ mla_status encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t r
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- projections
+// Token rows per projection launch (the kernel's N), and the padded N.
+constexpr int kProjMaxRows = 64;
+int proj_pad(int T) { return (std::min(T, kProjMaxRows) + 15) / 16 * 16; }
+int tiles_of(int rows) { return (rows + 127) / 128; }
+
+// Split of K over CTAs so that about four waves of CTAs stream the weights
+// (each CTA keeps at least 4 blocks of 64 columns).
+int proj_ksplit(int tiles, int K, int sm_count) {
+  const int kb = K / 64;
+  const int want = std::max(1, (4 * sm_count + tiles - 1) / tiles);
+  return std::max(1, std::min({want, kb / 4 > 0 ? kb / 4 : 1, 64}));
+}
+
+size_t proj_acc_bytes(int tiles) { return wgemm_workspace_bytes(tiles, kProjMaxRows); }
+
+mla_status encode_rows(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  return encode_2d(m, ptr, inner, rows, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// One projection over token rows [t0, t0 + n) of a call; the weight maps
+// and the epilogue arguments are filled in by the caller.
+mla_status run_projection(WgemmLaunch L, const void* X, int K, int T, int ldx_rows_per_token,
+                          const DeviceInfo* d, cudaStream_t s,
+                          const std::function<void(WgemmLaunch&, int t0)>& per_chunk) {
+  const int chunk = kProjMaxRows / ldx_rows_per_token;
+  for (int t0 = 0; t0 < T; t0 += chunk) {
+    const int n = std::min(chunk, T - t0) * ldx_rows_per_token;
+    WgemmLaunch C = L;
+    C.N = n;
+    C.n_pad = (n + 15) / 16 * 16;
+    const void* xp = static_cast<const uint8_t*>(X) + (size_t)t0 * ldx_rows_per_token * K * 2;
+    mla_status st = encode_2d(&C.x_map, xp, K, (uint64_t)n, 64, C.n_pad, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != MLA_OK) return st;
+    C.ksplit = proj_ksplit(C.tiles, K, d->sm_count);
+    per_chunk(C, t0);
+    if ((st = cuda_status(launch_wgemm(C, s))) != MLA_OK) return st;
+  }
+  return MLA_OK;
 }
 
 // 3D map over the queries [B * s_q, n_h, 576] (bf16), box box_x x 16 heads x 1.
@@ -421,7 +465,7 @@ mla_status mla_absorb_weights(const void* W_UK, const void* W_Q, void* W_QK, int
 
 mla_status mla_form_query(const void* h, const void* W_QK, const void* W_QR, const int* pos,
                           void* q, int T, int n_h, int d_model, int d_c, int d_R, float rope_base,
-                          mla_dtype dtype, void* stream) {
+                          mla_dtype dtype, void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dtype(dtype) || T < 0 || n_h < 1 || d_model < 1 || d_c < 1 || d_R < 0 || d_R % 2)
     return MLA_ERR_INVALID_ARG;
   if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
@@ -435,6 +479,34 @@ mla_status mla_form_query(const void* h, const void* W_QK, const void* W_QR, con
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int W = d_c + d_R;
+  if (dtype == MLA_DTYPE_BF16) {
+    // tensor cores: W = [W^QK (n_h * d_c rows) ; W^QR (n_h * d_R rows)]
+    if (!d->wgemm_tc || g_encode == nullptr) return MLA_ERR_UNSUPPORTED;
+    if (d_model % 64 != 0 || d_R % 2 != 0 || (d_R > 0 && 128 % d_R != 0)) return MLA_ERR_UNSUPPORTED;
+    const int rows0 = n_h * d_c, rows1 = n_h * d_R;
+    WgemmLaunch L = {};
+    L.tiles0 = tiles_of(rows0);
+    L.tiles = L.tiles0 + tiles_of(rows1);
+    if (workspace_bytes < proj_acc_bytes(L.tiles) || workspace == nullptr ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return workspace_bytes < proj_acc_bytes(L.tiles) ? MLA_ERR_WORKSPACE_TOO_SMALL : MLA_ERR_INVALID_ARG;
+    if ((st = encode_rows(&L.w_map[0], W_QK, d_model, rows0, 128)) != MLA_OK) return st;
+    L.w_map[1] = L.w_map[0];
+    if (rows1 > 0 && (st = encode_rows(&L.w_map[1], W_QR, d_model, rows1, 128)) != MLA_OK) return st;
+    L.K = d_model;
+    L.workspace = workspace;
+    L.err = d->flags;
+    L.mode = 3;
+    L.n_h = n_h;
+    L.d_c = d_c;
+    L.d_R = d_R;
+    L.rope_base = rope_base;
+    return run_projection(L, h, d_model, T, 1, d, s, [&](WgemmLaunch& C, int t0) {
+      C.out = static_cast<__nv_bfloat16*>(q) + (size_t)t0 * n_h * W;
+      C.pos = pos + t0;
+    });
+  }
+  // fp32 tensors: the tiled CUDA-core GEMM
   GemmArgs g = {};
   g.A = h;
   g.M = T;
@@ -472,7 +544,8 @@ mla_status mla_append_latent(const void* h, const void* W_DKV, const void* W_KR,
                              const int* seq_ids, const int* pos, const int* block_table,
                              int max_pages_per_seq, int page_size, int num_pages, void* kv_cache,
                              int T, int d_model, int d_c, int d_R, float rope_base,
-                             mla_dtype dtype, void* stream) {
+                             mla_dtype dtype, void* workspace, size_t workspace_bytes,
+                             void* stream) {
   if (!valid_dtype(dtype) || T < 0 || d_model < 1 || d_c < 1 || d_R < 0 || d_R % 2 ||
       page_size < 1 || max_pages_per_seq < 1 || num_pages < 1)
     return MLA_ERR_INVALID_ARG;
@@ -487,6 +560,37 @@ mla_status mla_append_latent(const void* h, const void* W_DKV, const void* W_KR,
   mla_status st = device_info(&d);
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == MLA_DTYPE_BF16) {
+    // tensor cores: W = [W^DKV (d_c rows) ; W^KR (d_R rows)]
+    if (!d->wgemm_tc || g_encode == nullptr) return MLA_ERR_UNSUPPORTED;
+    if (d_model % 64 != 0 || d_R % 2 != 0 || d_R > 128) return MLA_ERR_UNSUPPORTED;
+    WgemmLaunch L = {};
+    L.tiles0 = tiles_of(d_c);
+    L.tiles = L.tiles0 + tiles_of(d_R);
+    if (workspace_bytes < proj_acc_bytes(L.tiles) || workspace == nullptr ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return workspace_bytes < proj_acc_bytes(L.tiles) ? MLA_ERR_WORKSPACE_TOO_SMALL : MLA_ERR_INVALID_ARG;
+    if ((st = encode_rows(&L.w_map[0], W_DKV, d_model, d_c, 128)) != MLA_OK) return st;
+    L.w_map[1] = L.w_map[0];
+    if (d_R > 0 && (st = encode_rows(&L.w_map[1], W_KR, d_model, d_R, 128)) != MLA_OK) return st;
+    L.K = d_model;
+    L.workspace = workspace;
+    L.err = d->flags;
+    L.mode = 1;
+    L.out = kv_cache;
+    L.d_c = d_c;
+    L.d_R = d_R;
+    L.block_table = block_table;
+    L.max_pages = max_pages_per_seq;
+    L.page_size = page_size;
+    L.num_pages = num_pages;
+    L.rope_base = rope_base;
+    return run_projection(L, h, d_model, T, 1, d, s, [&](WgemmLaunch& C, int t0) {
+      C.pos = pos + t0;
+      C.seq = seq_ids + t0;
+    });
+  }
+  // fp32 tensors: the tiled CUDA-core GEMM
   GemmArgs g = {};
   g.A = h;
   g.C = kv_cache;
@@ -568,6 +672,137 @@ mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h,
       return MLA_ERR_CUDA;
   }
   return cuda_status(launch_up_proj_sm100(w_map, u_map, o, d->flags, T, n_h, d_c, d_v, f32, false, s));
+}
+
+mla_status mla_projection_workspace_size(int rows0, int rows1, int T, int x_fp32_K,
+                                         size_t* bytes) {
+  if (bytes == nullptr || rows0 < 0 || rows1 < 0 || T < 0 || x_fp32_K < 0) return MLA_ERR_INVALID_ARG;
+  size_t b = proj_acc_bytes(tiles_of(rows0) + tiles_of(rows1));
+  if (x_fp32_K > 0) b += align_up((size_t)2 * T * x_fp32_K * 2, 256);
+  *bytes = b;
+  return MLA_OK;
+}
+
+mla_status mla_form_query_fused(const void* h, const void* W_Q, const void* W_UK,
+                                const void* W_QR, const int* pos, void* q, int T, int n_h,
+                                int d_h, int d_model, int d_c, int d_R, float rope_base,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || n_h < 1 || d_h < 1 || d_model < 1 || d_c < 1 || d_R < 0 || d_R % 2)
+    return MLA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !W_Q || !W_UK || !q || (d_R > 0 && (!W_QR || !pos))) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(W_Q) || !aligned16(W_UK) || !aligned16(q) ||
+      (W_QR && !aligned16(W_QR)))
+    return MLA_ERR_INVALID_ARG;
+  // one 128-row tile per head of W^Q, whole heads of W^QR per tile, d_c in
+  // 128-row steps of the second product
+  if (d_h != 128 || d_c % 128 != 0 || d_c > 512 || d_model % 64 != 0 ||
+      (d_R > 0 && 128 % d_R != 0))
+    return MLA_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  if (!d->wgemm_tc || g_encode == nullptr) return MLA_ERR_UNSUPPORTED;
+  const int rows0 = n_h * d_h, rows1 = n_h * d_R;
+  WgemmLaunch L = {};
+  L.tiles0 = tiles_of(rows0);
+  L.tiles = L.tiles0 + tiles_of(rows1);
+  if (workspace_bytes < proj_acc_bytes(L.tiles)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MLA_ERR_INVALID_ARG;
+  if ((st = encode_rows(&L.w_map[0], W_Q, d_model, rows0, 128)) != MLA_OK) return st;
+  L.w_map[1] = L.w_map[0];
+  if (rows1 > 0 && (st = encode_rows(&L.w_map[1], W_QR, d_model, rows1, 128)) != MLA_OK) return st;
+  if ((st = encode_rows(&L.uk_map, W_UK, d_c, (uint64_t)n_h * d_h, 128)) != MLA_OK) return st;
+  L.K = d_model;
+  L.workspace = workspace;
+  L.err = d->flags;
+  L.mode = 0;
+  L.n_h = n_h;
+  L.d_c = d_c;
+  L.d_R = d_R;
+  L.rope_base = rope_base;
+  const int W = d_c + d_R;
+  return run_projection(L, h, d_model, T, 1, d, static_cast<cudaStream_t>(stream),
+                        [&](WgemmLaunch& C, int t0) {
+                          C.out = static_cast<__nv_bfloat16*>(q) + (size_t)t0 * n_h * W;
+                          C.pos = pos + t0;
+                        });
+}
+
+mla_status mla_fold_output_weights(const void* W_O, const void* W_UV, void* W_OUV, int n_h, int d_v,
+                                   int d_c, int d_model, mla_dtype dtype, void* stream) {
+  if (!W_O || !W_UV || !W_OUV || !valid_dtype(dtype)) return MLA_ERR_INVALID_ARG;
+  if (n_h < 1 || d_v < 1 || d_c < 1 || d_model < 1) return MLA_ERR_INVALID_ARG;
+  if (n_h > 65535) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(W_O) || !aligned16(W_UV) || !aligned16(W_OUV)) return MLA_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  // W_OUV[m][i * d_c + c] = sum_v W_O[m][i * d_v + v] W_UV[i][v][c]
+  GemmArgs g = {};
+  g.A = W_O;    // A(z = i, m, k = v) = W_O[m][i * d_v + v]
+  g.Bm = W_UV;  // B(z, n = c, k = v) = W_UV[i][v][c]
+  g.C = W_OUV;  // C(z, m, n) = W_OUV[m][i * d_c + n]
+  g.M = d_model;
+  g.N = d_c;
+  g.K = d_v;
+  g.Z = n_h;
+  g.sAz = d_v;
+  g.sAm = (long long)n_h * d_v;
+  g.sAk = 1;
+  g.sBz = (long long)d_v * d_c;
+  g.sBn = 1;
+  g.sBk = d_c;
+  g.sCz = d_c;
+  g.sCm = (long long)n_h * d_c;
+  g.seg = INT_MAX;
+  g.err = d->flags;
+  g.bf16 = dtype == MLA_DTYPE_BF16;
+  return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_output_projection(const void* x, mla_dtype x_dtype, const void* W, void* y, int T,
+                                 int K, int M, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!valid_dtype(x_dtype) || T < 0 || K < 1 || M < 1) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!x || !W || !y) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return MLA_ERR_INVALID_ARG;
+  if (K % 64 != 0 || M % 8 != 0) return MLA_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  if (!d->wgemm_tc || g_encode == nullptr) return MLA_ERR_UNSUPPORTED;
+  const bool f32 = x_dtype == MLA_DTYPE_FP32;
+  WgemmLaunch L = {};
+  L.tiles0 = L.tiles = tiles_of(M);
+  const size_t acc = proj_acc_bytes(L.tiles);
+  const size_t need = acc + (f32 ? align_up((size_t)2 * T * K * 2, 256) : 0);
+  if (workspace_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* X = x;
+  if (f32) {
+    // an fp32 x enters as two bf16 rows per token whose products are added
+    void* pairs = static_cast<uint8_t*>(workspace) + acc;
+    if ((st = cuda_status(launch_split_rows(static_cast<const float*>(x), pairs, T, K, s))) != MLA_OK)
+      return st;
+    X = pairs;
+  }
+  if ((st = encode_rows(&L.w_map[0], W, K, M, 128)) != MLA_OK) return st;
+  L.w_map[1] = L.w_map[0];
+  L.K = K;
+  L.workspace = workspace;
+  L.err = d->flags;
+  L.mode = 2;
+  L.ldo = M;
+  L.pair = f32 ? 2 : 1;
+  return run_projection(L, X, K, T, L.pair, d, s, [&](WgemmLaunch& C, int t0) {
+    C.out = static_cast<__nv_bfloat16*>(y) + (size_t)t0 * M;
+  });
 }
 
 mla_status mla_merge_partials(const void* u_parts, const float* lse_parts, void* u, float* lse,

@@ -125,6 +125,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;     // 2 x 128 columns
 constexpr uint32_t kTmemO = 256;   // 2 x 128 columns (latent blocks 0-255, 256-511)
 constexpr float kRescaleThreshold = 30.0f;  // log2 units: rescale O only if the max grows by > 2^30
+constexpr int kPrefetchAhead = 4;           // tiles between an L2 prefetch and the tile's TMA load
 constexpr uint16_t kBothCtas = 3;
 
 static_assert(kOffKv % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "align");
@@ -139,6 +140,7 @@ __device__ __forceinline__ int lat_col(int kc, int half) {
 struct Params {
   Sm100Maps maps;
   const __nv_bfloat16* q;  // [B * s_q, n_h, 576], for L2 prefetch of the next segment's rows
+  const __nv_bfloat16* kv; // the cache [rows, 576], for L2 prefetch of tiles ahead of their loads
   const int* block_table;
   const int* seqlens;
   const int* header;
@@ -280,6 +282,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n_here = min(32, sg.t1 - t0);
         for (int i = 0; i < n_here; ++i, ++g) {
           const int page = __shfl_sync(0xffffffffu, my_page, i);
+          // The tile kPrefetchAhead tiles later goes to L2 now: its TMA load is
+          // issued only when a stage frees (after this tile's P . C), and an
+          // L2 hit then lands in a fraction of the HBM latency, which would
+          // otherwise keep every stage busy that much longer.  A 64-token
+          // tile of one page is 64 x 1152 contiguous bytes; the even CTA
+          // fetches all of it.
+          // At the start of a chunk every SM is already loading its query and
+          // first stages; fetching more then only delays those, so the first
+          // kStages tiles of the chunk prefetch nothing.
+          const int page_ahead = __shfl_sync(0xffffffffu, my_page, (i + kPrefetchAhead) & 31);
+          if (leader && lane == 0 && g >= kStages && i + kPrefetchAhead < n_here) {
+            const int tok_a = (t0 + i + kPrefetchAhead) * kTileTokens;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(
+                p.kv + ((size_t)page_ahead * p.page_size + tok_a % p.page_size) * (kDc + 64));
+            constexpr uint32_t kTile = kTileTokens * (kDc + 64) * 2;
+            for (uint32_t off = 0; off < kTile; off += 16384)
+              bulk_prefetch_l2(src + off, min(16384u, kTile - off));
+          }
           if (lane == 0) {
             const int s = g % kStages, n = g / kStages;
             ok = mbar_wait(bar(KV_EMPTY + s), (n & 1) ^ 1, p.err, MLA_DEVFLAG_TIMEOUT);
@@ -852,6 +872,7 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   Params p;
   p.maps = maps;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.kv = static_cast<const __nv_bfloat16*>(a.kv);
   p.block_table = a.block_table;
   p.seqlens = a.seqlens;
   p.header = a.header;

@@ -161,5 +161,7 @@ struct WgemmLaunch {
 int wgemm_sm100_prepare();
 size_t wgemm_workspace_bytes(int tiles, int n_pad);
 cudaError_t launch_wgemm(const WgemmLaunch& L, cudaStream_t s);
+// x [T, K] fp32 -> pairs [2T, K] bf16 (hi, lo of every row)
+cudaError_t launch_split_rows(const float* x, void* pairs, int T, int K, cudaStream_t s);
 
 }  // namespace mla

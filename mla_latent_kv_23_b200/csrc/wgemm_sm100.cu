@@ -16,6 +16,9 @@
 //   kStore  ("Attention-head anatomy" section 5, W^UV folded into W^O):
 //            Y = W X written as y[t, m]; X may hold each token twice (two
 //            bf16 terms of an fp32 row), whose products are added.
+//   kQueryAbsorbed (absorption section, score equation, with the offline
+//            W^QK = W^UK^T W^Q): W = [W^QK ; W^QR], rows of W^QK_i give
+//            q[t, i, 0:d_c] directly, rows of W^QR as in kQuery.
 //
 // One CTA per (128-row tile of W, slice of K): M = 128, N = token rows
 // padded to 16, K streamed through a TMA pipeline of 64-column blocks with
@@ -25,6 +28,8 @@
 // to zero, so the workspace is zero again after every call.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "sm100_ptx.cuh"
@@ -57,7 +62,7 @@ struct Params {
   float* acc;            // [tiles][128][n_pad] fp32 workspace (zero on entry and exit)
   int* counters;         // [tiles]
   int* err;
-  int mode;              // 0 kQuery, 1 kCache, 2 kStore
+  int mode;              // 0 kQuery, 1 kCache, 2 kStore, 3 kQueryAbsorbed
   // kQuery: q [N, n_h, d_c + d_R]; kCache: the cache; kStore: y [N / pair, ldo]
   __nv_bfloat16* out;
   int n_h, d_c, d_R, ldo, pair;
@@ -208,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgemm_sm100_kernel(const __grid_c
       const int r = row0 + m;           // row within the RoPE tensor
       const int head = r / p.d_R, k = r % p.d_R;
       const int k2 = k & ~1;
-      const bool valid = p.mode == 0 ? head < p.n_h : r < p.d_R;
+      const bool valid = p.mode != 1 ? head < p.n_h : r < p.d_R;
       for (int t = 0; t < p.N; ++t) {
         const float x = vals[t];
         const float y = __shfl_xor_sync(0xffffffffu, x, 1);
@@ -217,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgemm_sm100_kernel(const __grid_c
         rope_cs(p.pos[t], k2, p.d_R, p.log_base, c, s);
         // (x_even, x_odd) -> (x_even c - x_odd s, x_even s + x_odd c)
         const float out = (k & 1) ? (y * s + x * c) : (x * c - y * s);
-        if (p.mode == 0) {
+        if (p.mode != 1) {
           p.out[((size_t)t * p.n_h + head) * (p.d_c + p.d_R) + p.d_c + k] = __float2bfloat16_rn(out);
         } else {
           const int pg_i = p.pos[t] / p.page_size;
@@ -230,6 +235,12 @@ __global__ void __launch_bounds__(kThreads, 1) wgemm_sm100_kernel(const __grid_c
           p.out[crow * (p.d_c + p.d_R) + p.d_c + k] = __float2bfloat16_rn(out);
         }
       }
+    } else if (p.mode == 3) {
+      // rows (head, c) of the flattened W^QK: q[t, head, c]
+      const int r = row0 + m, head = r / p.d_c, c = r % p.d_c;
+      if (head < p.n_h)
+        for (int t = 0; t < p.N; ++t)
+          p.out[((size_t)t * p.n_h + head) * (p.d_c + p.d_R) + c] = __float2bfloat16_rn(vals[t]);
     } else if (p.mode == 1) {
       // latent rows c = row0 + m of the new tokens' cache rows
       const int c = row0 + m;
@@ -339,6 +350,28 @@ int wgemm_sm100_prepare() {
 
 size_t wgemm_workspace_bytes(int tiles, int n_pad) {
   return ((size_t)tiles * 128 * n_pad * sizeof(float) + 255) / 256 * 256 + (size_t)tiles * sizeof(int);
+}
+
+// fp32 rows -> pairs of bf16 rows: pairs[2t] = bf16(x[t]), pairs[2t + 1] =
+// bf16(x[t] - pairs[2t]); the two terms add back to x within 2^-16 of it.
+__global__ void split_rows_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ pairs,
+                                  int T, int K) {
+  const size_t n = (size_t)T * K;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t t = i / K, k = i % K;
+    const float v = x[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    pairs[(2 * t) * K + k] = hi;
+    pairs[(2 * t + 1) * K + k] = __float2bfloat16_rn(v - __bfloat162float(hi));
+  }
+}
+
+cudaError_t launch_split_rows(const float* x, void* pairs, int T, int K, cudaStream_t s) {
+  const size_t n = (size_t)T * K;
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
+  split_rows_kernel<<<blocks, 256, 0, s>>>(x, static_cast<__nv_bfloat16*>(pairs), T, K);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wgemm(const WgemmLaunch& L, cudaStream_t s) {

@@ -45,8 +45,13 @@ _P = ctypes.POINTER(DecodeParams)
 SIGNATURES = {
     "mla_status_string": ([_I], ctypes.c_char_p),
     "mla_absorb_weights": ([_V, _V, _V, _I, _I, _I, _I, _I, _V], _I),
-    "mla_form_query": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _I, _V], _I),
-    "mla_append_latent": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _V, _I, _I, _I, _I, _F, _I, _V], _I),
+    "mla_projection_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_S)], _I),
+    "mla_form_query": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _I, _V, _S, _V], _I),
+    "mla_form_query_fused": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _F, _V, _S, _V], _I),
+    "mla_append_latent": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _V, _I, _I, _I, _I, _F, _I, _V, _S,
+                           _V], _I),
+    "mla_fold_output_weights": ([_V, _V, _V, _I, _I, _I, _I, _I, _V], _I),
+    "mla_output_projection": ([_V, _I, _V, _V, _I, _I, _I, _V, _S, _V], _I),
     "mla_decode_workspace_size": ([_P, ctypes.POINTER(_S)], _I),
     "mla_decode": ([_P, _V, _S, _V], _I),
     "mla_decode_plan": ([_P, _V, _S, _V], _I),
@@ -129,27 +134,92 @@ def mla_absorb_weights(W_UK, W_Q, W_QK, stream=None) -> None:
                                     _dtype_code(W_UK), _stream(stream)), "mla_absorb_weights")
 
 
-def mla_form_query(h, W_QK, W_QR, pos, q, rope_base: float = 10000.0, stream=None) -> None:
+def mla_projection_workspace_size(rows0: int, rows1: int, T: int, x_fp32_K: int = 0) -> int:
+    n = _S(0)
+    _check(lib().mla_projection_workspace_size(rows0, rows1, T, x_fp32_K, ctypes.byref(n)),
+           "mla_projection_workspace_size")
+    return n.value
+
+
+def projection_workspace(rows0: int, rows1: int, T: int, device, x_fp32_K: int = 0):
+    """A zeroed projection workspace (the calls leave it zero again)."""
+    torch = _torch()
+    n = mla_projection_workspace_size(rows0, rows1, T, x_fp32_K)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def _ws(ws):
+    return (None, 0) if ws is None else (_ptr(ws), ws.numel() * ws.element_size())
+
+
+def mla_form_query(h, W_QK, W_QR, pos, q, rope_base: float = 10000.0, workspace=None,
+                   stream=None) -> None:
+    """q [T, n_h, d_c + d_R] = [W_QK h || RoPE(W_QR h, pos)]; bf16 needs a
+    projection workspace (one is made if none is given)."""
     T, d_model = h.shape
     n_h, d_c, _ = W_QK.shape
     d_R = W_QR.shape[1]
     assert q.shape == (T, n_h, d_c + d_R)
+    if workspace is None and _dtype_code(h) == MLA_DTYPE_BF16:
+        workspace = projection_workspace(n_h * d_c, n_h * d_R, T, h.device)
+    wp, wn = _ws(workspace)
     _check(lib().mla_form_query(_ptr(h), _ptr(W_QK), _ptr(W_QR), _ptr(pos), _ptr(q), T, n_h,
-                                d_model, d_c, d_R, float(rope_base), _dtype_code(h),
+                                d_model, d_c, d_R, float(rope_base), _dtype_code(h), wp, wn,
                                 _stream(stream)), "mla_form_query")
 
 
+def mla_form_query_fused(h, W_Q, W_UK, W_QR, pos, q, rope_base: float = 10000.0, workspace=None,
+                         stream=None) -> None:
+    """q = [W_UK^T (W_Q h) || RoPE(W_QR h, pos)] without a precomputed W_QK."""
+    T, d_model = h.shape
+    n_h, d_h, d_c = W_UK.shape
+    d_R = W_QR.shape[1]
+    assert W_Q.shape == (n_h, d_h, d_model) and q.shape == (T, n_h, d_c + d_R)
+    if workspace is None:
+        workspace = projection_workspace(n_h * d_h, n_h * d_R, T, h.device)
+    wp, wn = _ws(workspace)
+    _check(lib().mla_form_query_fused(_ptr(h), _ptr(W_Q), _ptr(W_UK), _ptr(W_QR), _ptr(pos),
+                                      _ptr(q), T, n_h, d_h, d_model, d_c, d_R, float(rope_base),
+                                      wp, wn, _stream(stream)), "mla_form_query_fused")
+
+
 def mla_append_latent(h, W_DKV, W_KR, seq_ids, pos, block_table, kv_cache, page_size: int,
-                      rope_base: float = 10000.0, stream=None) -> None:
+                      rope_base: float = 10000.0, workspace=None, stream=None) -> None:
     T, d_model = h.shape
     d_c, d_R = W_DKV.shape[0], W_KR.shape[0]
     rows, width = kv_cache.shape
     assert width == d_c + d_R and rows % page_size == 0
+    if workspace is None and _dtype_code(h) == MLA_DTYPE_BF16:
+        workspace = projection_workspace(d_c, d_R, T, h.device)
+    wp, wn = _ws(workspace)
     _check(lib().mla_append_latent(_ptr(h), _ptr(W_DKV), _ptr(W_KR), _ptr(seq_ids), _ptr(pos),
                                    _ptr(block_table), block_table.shape[1], page_size,
                                    rows // page_size, _ptr(kv_cache), T, d_model, d_c, d_R,
-                                   float(rope_base), _dtype_code(h), _stream(stream)),
+                                   float(rope_base), _dtype_code(h), wp, wn, _stream(stream)),
            "mla_append_latent")
+
+
+def mla_fold_output_weights(W_O, W_UV, W_OUV, stream=None) -> None:
+    """W_OUV [d_model, n_h * d_c] = W_O [d_model, n_h * d_v] . blockdiag(W_UV [n_h, d_v, d_c])."""
+    n_h, d_v, d_c = W_UV.shape
+    d_model = W_O.shape[0]
+    assert W_O.shape == (d_model, n_h * d_v) and W_OUV.shape == (d_model, n_h * d_c)
+    _check(lib().mla_fold_output_weights(_ptr(W_O), _ptr(W_UV), _ptr(W_OUV), n_h, d_v, d_c,
+                                         d_model, _dtype_code(W_O), _stream(stream)),
+           "mla_fold_output_weights")
+
+
+def mla_output_projection(x, W, y, workspace=None, stream=None) -> None:
+    """y [T, M] = x [T, K] . W [M, K]^T (W bf16; x bf16 or float32)."""
+    T, K = x.shape
+    M = W.shape[0]
+    assert W.shape == (M, K) and y.shape == (T, M)
+    f32 = _dtype_code(x) == MLA_DTYPE_FP32
+    if workspace is None:
+        workspace = projection_workspace(M, 0, T, x.device, K if f32 else 0)
+    wp, wn = _ws(workspace)
+    _check(lib().mla_output_projection(_ptr(x), _dtype_code(x), _ptr(W), _ptr(y), T, K, M, wp, wn,
+                                       _stream(stream)), "mla_output_projection")
 
 
 def decode_params(q, kv_cache, block_table, seqlens, u, lse, page_size: int, d_R: int,

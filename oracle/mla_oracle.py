@@ -287,6 +287,29 @@ def decode_absorbed_seq(q_b: np.ndarray, cache, block_table, L: int, b: int, w,
     return (u, lse, abs_c) if want_abs else (u, lse)
 
 
+def absorbed_queries_all(inp: dict, w) -> np.ndarray:
+    """absorbed_queries for every (b, r): [B, s_q, n_h, d_c + d_R].  The same
+    two products per head, W^UK_i^T (W^Q_i h) and RoPE(W^QR_i h, pos), taken
+    over all query rows at once."""
+    H = np.asarray(inp["h_q"], f64).reshape(w.B * w.s_q, w.d_model)             # [T, d_model]
+    qn = np.tensordot(H, np.asarray(inp["W_Q"], f64), axes=([1], [2]))          # [T, n_h, d_h]
+    qlat = np.einsum("thk,hkc->thc", qn, np.asarray(inp["W_UK"], f64))          # [T, n_h, d_c]
+    qr = np.tensordot(H, np.asarray(inp["W_QR"], f64), axes=([1], [2]))         # [T, n_h, d_R]
+    pos = np.asarray(inp["qpos"]).reshape(-1)
+    for t in range(qr.shape[0]):
+        qr[t] = np.stack([rope(x, int(pos[t]), w.rope_base) for x in qr[t]])
+    return np.concatenate([qlat, qr], axis=2).reshape(w.B, w.s_q, w.n_h, w.d_c + w.d_R)
+
+
+def output_projection(o: np.ndarray, W_O: np.ndarray) -> np.ndarray:
+    """y_t = W^O concat_i(o_{t,i}): the heads' outputs concatenated and
+    projected to the hidden size ("Attention-head anatomy" section 5, the
+    output side W^O that W^UV folds into).  o [T, n_h, d_v],
+    W^O [d_model, n_h * d_v] -> y [T, d_model]."""
+    o = np.asarray(o, f64)
+    return o.reshape(o.shape[0], -1) @ np.asarray(W_O, f64).T
+
+
 def up_project(u: np.ndarray, W_UV: np.ndarray) -> np.ndarray:
     """o_i = W^UV_i u_i: u [..., n_h, d_c], W^UV [n_h, d_v, d_c] -> [..., n_h, d_v]."""
     return np.einsum("...hc,hvc->...hv", np.asarray(u, f64), np.asarray(W_UV, f64))

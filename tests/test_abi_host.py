@@ -89,13 +89,33 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.mla_up_proj(16, 32, 48, 4, 128, 512, 128, 3, 0, None) == INVALID  # u dtype
     assert lib.mla_up_proj(16, 32, 48, 4, 128, 512, 129, 1, 0, None) == UNSUPPORTED  # d_v > 128
     assert lib.mla_up_proj(16, 32, 48, 4, 128, 96, 128, 1, 0, None) == UNSUPPORTED   # bf16 d_c % 64
-    assert lib.mla_form_query(16, 32, 48, 64, 80, 4, 128, 7168, 512, 63, 1e4, 0, None) == INVALID
-    assert lib.mla_form_query(16, 32, 48, 64, 80, 4, 128, 7168, 512, 64, -1.0, 0, None) == INVALID
-    assert lib.mla_form_query(16, 32, 48, 64, 80, 0, 128, 7168, 512, 64, 1e4, 0, None) == OK
+    assert lib.mla_form_query(16, 32, 48, 64, 80, 4, 128, 7168, 512, 63, 1e4, 0, None, 0,
+                              None) == INVALID
+    assert lib.mla_form_query(16, 32, 48, 64, 80, 4, 128, 7168, 512, 64, -1.0, 0, None, 0,
+                              None) == INVALID
+    assert lib.mla_form_query(16, 32, 48, 64, 80, 0, 128, 7168, 512, 64, 1e4, 0, None, 0,
+                              None) == OK
     assert lib.mla_append_latent(16, 32, 48, 64, 80, 96, 4, 0, 8, 112, 4, 256, 64, 16, 1e4, 0,
-                                 None) == INVALID
+                                 None, 0, None) == INVALID
     assert lib.mla_append_latent(16, 32, 48, 64, 80, 96, 4, 64, 8, None, 4, 256, 64, 16, 1e4, 0,
-                                 None) == INVALID
+                                 None, 0, None) == INVALID
+    # fused query formation: odd d_R, null weights, and shapes outside the kernel
+    assert lib.mla_form_query_fused(16, 32, 48, 64, 80, 96, 4, 128, 128, 7168, 512, 63, 1e4,
+                                    None, 0, None) == INVALID
+    assert lib.mla_form_query_fused(16, None, 48, 64, 80, 96, 4, 128, 128, 7168, 512, 64, 1e4,
+                                    None, 0, None) == INVALID
+    assert lib.mla_form_query_fused(16, 32, 48, 64, 80, 96, 4, 128, 64, 7168, 512, 64, 1e4,
+                                    None, 0, None) == UNSUPPORTED          # d_h != 128
+    assert lib.mla_form_query_fused(16, 32, 48, 64, 80, 96, 0, 128, 128, 7168, 512, 64, 1e4,
+                                    None, 0, None) == OK                   # T = 0
+    # output projection: K not a multiple of 64; fold: null weights
+    assert lib.mla_output_projection(16, 0, 32, 48, 4, 100, 7168, None, 0, None) == UNSUPPORTED
+    assert lib.mla_output_projection(16, 5, 32, 48, 4, 128, 7168, None, 0, None) == INVALID
+    assert lib.mla_fold_output_weights(None, 32, 48, 128, 128, 512, 7168, 0, None) == INVALID
+    n = ctypes.c_size_t(0)
+    assert lib.mla_projection_workspace_size(16384, 8192, 16, 0, ctypes.byref(n)) == OK
+    assert n.value >= (128 + 64) * 128 * 64 * 4
+    assert lib.mla_projection_workspace_size(-1, 0, 16, 0, ctypes.byref(n)) == INVALID
 
 
 def test_binding_refuses_host_tensors():

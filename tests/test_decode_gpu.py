@@ -121,9 +121,22 @@ def test_small_latent_on_exact_inputs(dtype):
     out = run_pipeline(w, inp, num_splits=7, q=to_dev(q, w))
     picks = [(b, r, i) for b in range(w.B) for r in range(w.s_q) for i in range(w.n_h)]
     res = check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"])
-    assert_parity(res)
     if dtype == "bf16":
         assert_tight(res)
+        return
+    # fp32 tensors run as tf32 (10 stored significand bits): every product of
+    # a score carries up to 2^-10 of each operand, so an lse (a smooth maximum
+    # of scale * scores) can move by up to scale * 2^-9 * max_j sum_k |q_k c_jk|,
+    # more than 1e-3 of an lse near 0; lse is held to the larger of the two
+    assert res["o"] <= ATOL_REL and res["u"] <= ATOL_REL, res
+    lse = f64(out["lse"])
+    ref = orc.decode_absorbed(q, inp["cache"], inp["block_table"], inp["seqlens"], w, picks)
+    for (b, r, i), (_, lse_ref) in ref.items():
+        L = int(inp["seqlens"][b])
+        rows = orc.gather_rows(inp["cache"], inp["block_table"], w.page_size, b, L - w.s_q + r + 1)
+        tf32 = w.softmax_scale * 2.0 ** -9 * float(np.max(np.abs(rows) @ np.abs(q[b, r, i])))
+        allow = max(1e-3 * max(abs(lse_ref), 1.0), tf32)
+        assert abs(lse[b, r, i] - lse_ref) <= allow, (b, r, i, lse[b, r, i], lse_ref, allow)
 
 
 def test_unsupported_latent_widths_are_refused():

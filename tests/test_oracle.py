@@ -139,6 +139,40 @@ def test_all_heads_helpers_reproduce_the_expanded_definition(s_q):
     assert _max_abs(abs_c, u) < 1e-12
 
 
+def test_batched_queries_reproduce_the_expanded_definition():
+    # absorbed_queries_all (all rows at once) through the absorbed decode
+    # gives the expanded oracle's o and lse
+    w = medium_workload()
+    inp = synth.draw(w)
+    qa = orc.absorbed_queries_all(inp, w)
+    ua = orc.decode_absorbed(qa, inp["cache"], inp["block_table"], inp["seqlens"], w)
+    for key, (o, lse) in orc.decode_expanded(inp, w).items():
+        u, lse_a = ua[key]
+        assert _max_abs(orc.up_project(u[None, :], inp["W_UV"][key[2]][None])[0], o) < 1e-10
+        assert abs(lse_a - lse) < 1e-10
+
+
+def test_output_projection_brute_force():
+    # y_t[m] = sum over heads i and value dims v of W_O[m, i d_v + v] o_t[i, v],
+    # summed term by term with math.fsum
+    rng = np.random.default_rng(8)
+    T, n_h, d_v, d_model = 3, 4, 5, 7
+    o = rng.standard_normal((T, n_h, d_v))
+    W_O = rng.standard_normal((d_model, n_h * d_v))
+    y = orc.output_projection(o, W_O)
+    for t in range(T):
+        for m in range(d_model):
+            ref = math.fsum(W_O[m, i * d_v + v] * o[t, i, v] for i in range(n_h) for v in range(d_v))
+            assert abs(y[t, m] - ref) < 1e-12 * (1 + abs(ref))
+    # heads are concatenated in order: moving one head's values moves the
+    # contribution to that head's columns of W_O only
+    o2 = o.copy()
+    o2[:, 1] = 0.0
+    W2 = W_O.copy()
+    W2[:, d_v:2 * d_v] = 0.0
+    assert _max_abs(orc.output_projection(o2, W_O), orc.output_projection(o, W2)) < 1e-12
+
+
 def test_absorbed_scores_equal_expanded_scores():
     rng = np.random.default_rng(3)
     n_h, d_h, d_c, d_model = 3, 5, 7, 11
