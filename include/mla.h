@@ -254,6 +254,41 @@ mla_status mla_decode_kernel_info(const mla_decode_params* p, int* uses_tensor_c
                                   int* num_chunks);
 
 /*
+ * GQLA's GQA path (GQLA summary, abstract and method paragraphs: the same
+ * trained weights expose, besides the MQA-absorb path above, a GQA path with
+ * a per-group expanded cache; heads of a group share W^UK_g and W^UV_g).  A
+ * cached token holds, for each group g, K^C_g = W^UK_g c and V_g = W^UV_g c,
+ * and once the RoPE key k^R shared by all heads.  For head i of group
+ * g = i / (n_h / n_g), query row r < s_q of sequence b:
+ *   s_j = q[b,r,i,:d_h] . K^C_g[j] + q[b,r,i,d_h:] . k^R[j]   for j <= seqlens[b] - s_q + r
+ *   o[b,r,i,:] = sum_j softmax(softmax_scale * s)_j V_g[j];  lse as in mla_decode
+ * One CTA takes a KV chunk of one group with all its heads and all s_q query
+ * rows as the MMA rows, so the group's cache is read once for both rows of
+ * multi-token prediction (s_q = 2).  bf16 on the tensor cores; chunks and
+ * their merge as in mla_decode (fp32 partials).
+ */
+typedef struct {
+  const void* q;            /* [B, s_q, n_h, d_h + d_R] device: q^nope then q^R            */
+  const void* kv;           /* [num_pages * page_size, n_g, d_h + d_v] device: K^C_g then V_g */
+  const void* k_rope;       /* [num_pages * page_size, d_R] device                         */
+  const int* block_table;   /* [B, max_pages_per_seq] int32 device                         */
+  const int* seqlens;       /* [B] int32 device                                            */
+  void* o;                  /* [B, s_q, n_h, d_v] device, written (bf16, or fp32 if o_fp32) */
+  float* lse;               /* [B, s_q, n_h] fp32 device, written; may be NULL             */
+  int B, s_q, n_h, n_g;     /* s_q in {1, 2}; n_h a multiple of n_g; (n_h / n_g) s_q <= 128 */
+  int d_h, d_v, d_R;        /* d_h, d_v multiples of 64; d_h + d_R <= 256; d_v <= 256      */
+  int page_size, max_pages_per_seq, num_pages;
+  float softmax_scale;
+  mla_dtype dtype;          /* MLA_DTYPE_BF16                                              */
+  int num_splits;           /* KV chunks; 0 = automatic                                    */
+  int o_fp32;
+} mla_gqa_params;
+
+mla_status mla_decode_gqa_workspace_size(const mla_gqa_params* p, size_t* bytes);
+mla_status mla_decode_gqa(const mla_gqa_params* p, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
  * Per-head up-projection ("MLA deep compression", absorption section, output
  * equation):  o[t, i, :] = W_UV[i] . u[t, i, :]
  *   u     [T, n_h, d_c]   device, read   (T = B * s_q), type u_dtype

@@ -674,6 +674,126 @@ mla_status mla_up_proj(const void* u, const void* W_UV, void* o, int T, int n_h,
   return cuda_status(launch_up_proj_sm100(w_map, u_map, o, d->flags, T, n_h, d_c, d_v, f32, false, s));
 }
 
+namespace {
+
+mla_status validate_gqa(const mla_gqa_params* p) {
+  if (p == nullptr) return MLA_ERR_INVALID_ARG;
+  if (p->B < 0 || p->s_q < 1 || p->n_h < 1 || p->n_g < 1 || p->d_h < 1 || p->d_v < 1 || p->d_R < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (p->s_q > 2 || p->n_h % p->n_g != 0) return p->s_q > 2 ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+  if (p->page_size <= 0 || p->page_size % kTileTokens != 0) return MLA_ERR_INVALID_ARG;
+  if (p->max_pages_per_seq < 1 || p->num_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale) || !(p->softmax_scale > 0.f)) return MLA_ERR_INVALID_ARG;
+  if (p->d_R % 8 != 0 || p->num_splits < 0) return MLA_ERR_INVALID_ARG;
+  if (p->dtype != MLA_DTYPE_BF16) return valid_dtype(p->dtype) ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+  if (p->d_h % 64 != 0 || p->d_v % 64 != 0 || p->d_h + p->d_R > 256 || p->d_v > 256 ||
+      (p->n_h / p->n_g) * p->s_q > 128)
+    return MLA_ERR_UNSUPPORTED;
+  if ((long long)p->num_pages * p->page_size > INT_MAX ||
+      (long long)p->max_pages_per_seq * p->page_size > INT_MAX)
+    return MLA_ERR_UNSUPPORTED;
+  if (p->B == 0) return MLA_OK;
+  if (!p->q || !p->kv || (p->d_R > 0 && !p->k_rope) || !p->block_table || !p->seqlens || !p->o)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(p->q) || !aligned16(p->kv) || (p->k_rope && !aligned16(p->k_rope)) ||
+      !aligned16(p->o) || !aligned16(p->block_table) || !aligned16(p->seqlens) ||
+      (p->lse && !aligned16(p->lse)))
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+int gqa_chunks(const mla_gqa_params* p, const DeviceInfo* d) {
+  if (p->num_splits > 0) return p->num_splits;
+  return std::max(1, d->sm_count / p->n_g);  // one CTA per SM
+}
+
+}  // namespace
+
+mla_status mla_decode_gqa_workspace_size(const mla_gqa_params* p, size_t* bytes) {
+  if (bytes == nullptr) return MLA_ERR_INVALID_ARG;
+  mla_status st = validate_gqa(p);
+  if (st != MLA_OK) return st;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  *bytes = ws_layout(p->B, p->s_q, p->n_h, p->d_v, gqa_chunks(p, d)).total;
+  return MLA_OK;
+}
+
+mla_status mla_decode_gqa(const mla_gqa_params* p, void* ws, size_t ws_bytes, void* stream) {
+  mla_status st = validate_gqa(p);
+  if (st != MLA_OK || p->B == 0) return st;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != MLA_OK) return st;
+  if (d->cc_major != 10 || !d->small_tc || g_encode == nullptr) return MLA_ERR_UNSUPPORTED;
+  const int G = gqa_chunks(p, d);
+  const WsLayout L = ws_layout(p->B, p->s_q, p->n_h, p->d_v, G);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MLA_ERR_INVALID_ARG;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  DecodeArgs a = {};
+  a.q = p->q;
+  a.kv = p->kv;
+  a.block_table = p->block_table;
+  a.seqlens = p->seqlens;
+  a.u = p->o;
+  a.lse = p->lse;
+  a.header = reinterpret_cast<int*>(w + L.header);
+  a.tile_prefix = reinterpret_cast<int*>(w + L.tile_prefix);
+  a.split_base = reinterpret_cast<int*>(w + L.split_base);
+  a.chunk_t = reinterpret_cast<int*>(w + L.chunk_t);
+  a.chunk_b = reinterpret_cast<int*>(w + L.chunk_b);
+  a.part_lse = reinterpret_cast<float*>(w + L.part_lse);
+  a.part_u = reinterpret_cast<float*>(w + L.part_u);
+  a.err = d->flags;
+  a.B = p->B;
+  a.s_q = p->s_q;
+  a.n_h = p->n_h;
+  a.d_c = p->d_v;  // output width for the attend epilogue and the combine
+  a.d_R = p->d_R;
+  a.page_size = p->page_size;
+  a.max_pages = p->max_pages_per_seq;
+  a.num_pages = p->num_pages;
+  a.num_chunks = G;
+  a.scale = p->softmax_scale;
+  a.bf16 = true;
+  a.out_f32 = p->o_fp32 != 0;
+  a.part_bf16 = false;
+  a.pdl = false;
+  const int hpg = p->n_h / p->n_g;
+  const uint64_t wq = (uint64_t)p->d_h + p->d_R, wkv = (uint64_t)p->d_h + p->d_v;
+  const uint64_t rows = (uint64_t)p->num_pages * p->page_size;
+  CUtensorMap q_map, kv_map, kr_map;
+  memset(&kr_map, 0, sizeof(kr_map));
+  {
+    const cuuint64_t dims[3] = {wq, (cuuint64_t)p->n_h, (cuuint64_t)p->B * p->s_q};
+    const cuuint64_t strides[2] = {wq * 2, (cuuint64_t)p->n_h * wq * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)hpg, (cuuint32_t)p->s_q};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (g_encode(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p->q), dims, strides,
+                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {wkv, (cuuint64_t)p->n_g, rows};
+    const cuuint64_t strides[2] = {wkv * 2, (cuuint64_t)p->n_g * wkv * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kTileTokens};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (g_encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p->kv), dims,
+                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  if (p->d_R > 0 && (st = encode_2d(&kr_map, p->k_rope, p->d_R, rows, 64, kTileTokens,
+                                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_status(launch_plan(a, s))) != MLA_OK) return st;
+  const GqaShape gs{p->n_g, p->d_h, p->d_v, p->d_R};
+  if ((st = cuda_status(launch_decode_gqa_sm100(a, gs, q_map, kv_map, kr_map, s))) != MLA_OK) return st;
+  return cuda_status(launch_combine(a, s));
+}
+
 mla_status mla_projection_workspace_size(int rows0, int rows1, int T, int x_fp32_K,
                                          size_t* bytes) {
   if (bytes == nullptr || rows0 < 0 || rows1 < 0 || T < 0 || x_fp32_K < 0) return MLA_ERR_INVALID_ARG;

@@ -29,6 +29,15 @@
 // P is rounded to the operand type before it is stored (tf32 or bf16), and
 // u is normalised by the sum of the rounded weights it was built from; lse
 // uses the unrounded ones.
+//
+// The same kernel runs the GQA path of GQLA (GQLA summary, abstract and
+// method paragraphs: the same weights expose a path with a per-group expanded
+// cache).  There a cached token holds, for every group g of heads, the
+// expanded key K^C_g = W^UK_g c and value V_g = W^UV_g c, plus the RoPE key
+// shared by all heads; one CTA takes (KV chunk, group) with every head of the
+// group and every query row as the MMA rows, so a tile of the group's cache
+// is read once for all s_q rows (the MTP case, s_q = 2).  S is taken over
+// [K^C_g || k^R] and P . V over V_g, loaded into the stage's value region.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -64,8 +73,11 @@ enum Bar {
 
 struct Params {
   CUtensorMap q_map;   // q [B * s_q, n_h, W]: box (one 128-byte block) x 128 heads x 1
+                       // (GQA: box (one block) x heads per group x s_q)
   CUtensorMap kv_map;  // cache [rows, W]: box (one 128-byte block) x 64 rows
+                       // (GQA: the expanded cache [rows, n_g, d_h + d_v], box 64 x 1 x 64)
   CUtensorMap kv_pv_map;  // tf32: the same boxes with 32-byte-atom swizzle (P . C operand)
+  CUtensorMap kr_map;  // GQA: the shared RoPE keys [rows, d_R], box 64 x 64 rows
   const int* block_table;
   const int* seqlens;
   const int* header;
@@ -79,23 +91,26 @@ struct Params {
   float* part_lse;
   int* err;
   int B, s_q, n_h, d_c, max_pages, page_size, num_pages;
-  int blocks;          // 128-byte column blocks per cached row
+  int blocks;          // 128-byte column blocks of the S operand
   int out_f32;         // u is fp32 (else bf16)
   float scale_log2;    // softmax_scale * log2(e)
+  // GQA path: groups, heads per group, key / value / RoPE blocks
+  int n_g, hpg, d_h, d_v, nbk, nbr, nbv;
 };
 
-template <bool kTf32>
+template <bool kTf32, bool kGqa>
 struct Layout {
   static constexpr int kCols = kTf32 ? 32 : 64;          // values per 128-byte block
   static constexpr int kPBlocks = kTf32 ? 2 : 1;         // P: 64 tokens per row
-  static constexpr int kStages = kTf32 ? 2 : 3;
+  static constexpr bool kValueRegion = kTf32 || kGqa;    // P . C / P . V operand apart
+  static constexpr int kStages = kValueRegion ? 2 : 3;
   static constexpr int kPSlots = kTf32 ? 1 : 2;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKv = kOffQ + kMaxBlocks * kQBlkBytes;
-  // a stage: the S copy of the tile, then (tf32) the P . C copy of its
-  // latent columns
+  // a stage: the S operand of the tile, then (tf32, GQA) the value region:
+  // the P . C copy of the latent columns, or the group's values
   static constexpr uint32_t kPvCopy = kMaxBlocks * kKvBlkBytes;
-  static constexpr uint32_t kStageBytes = (kTf32 ? 2 : 1) * kMaxBlocks * kKvBlkBytes;
+  static constexpr uint32_t kStageBytes = (kValueRegion ? 2 : 1) * kMaxBlocks * kKvBlkBytes;
   static constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;
   static constexpr uint32_t kPSlot = kPBlocks * kQBlkBytes;
   static constexpr uint32_t kOffBar = kOffP + kPSlots * kPSlot;
@@ -110,9 +125,9 @@ __device__ __forceinline__ float to_tf32(float x) {
   return __uint_as_float(r);
 }
 
-template <bool kTf32>
+template <bool kTf32, bool kGqa>
 __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const __grid_constant__ Params p) {
-  using Lay = Layout<kTf32>;
+  using Lay = Layout<kTf32, kGqa>;
   constexpr int kStages = Lay::kStages;
   constexpr int kPSlots = Lay::kPSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -120,11 +135,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (sbase - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x / p.s_q, qrow = blockIdx.x % p.s_q;
+  // MLA: (chunk, query row); GQA: (chunk, group) with every query row
+  const int chunk = blockIdx.x / (kGqa ? p.n_g : p.s_q);
+  const int qrow = kGqa ? 0 : blockIdx.x % p.s_q;
+  const int grp = kGqa ? blockIdx.x % p.n_g : 0;
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kOffBar + 8u * i; };
   const int nb = p.blocks;
-  const int d_c = p.d_c;
-  const int nbc = kTf32 ? d_c / Lay::kCols : 0;  // blocks of the P . C copy
+  const int d_c = kGqa ? p.d_v : p.d_c;  // width of O and of the output rows
+  const int nbc = kGqa ? p.nbv : kTf32 ? d_c / Lay::kCols : 0;  // value-region blocks
+  const int q_rows = kGqa ? p.hpg * p.s_q : kRows;               // query rows the TMA fills
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -147,6 +166,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
     tmem_alloc(sbase + Lay::kOffTmemSlot, 512);
     tmem_relinquish();
   }
+  if (kGqa) {
+    // the query boxes fill rows [0, hpg * s_q) of each block; the rows past
+    // them are zero once and stay so
+    for (uint32_t off = threadIdx.x * 16; off < kMaxBlocks * kQBlkBytes; off += kThreads * 16)
+      *reinterpret_cast<uint4*>(base + Lay::kOffQ + off) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -161,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
       prefetch_tmap(&p.q_map);
       prefetch_tmap(&p.kv_map);
       if (kTf32) prefetch_tmap(&p.kv_pv_map);
+      if (kGqa) prefetch_tmap(&p.kr_map);
       ChunkWalk walk;
       walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
       Segment sg;
@@ -170,10 +197,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
         // the query area is free once the previous segment's last S is done
         if (seg_i > 0 && !(ok = mbar_wait(bar(Q_EMPTY), (seg_i - 1) & 1, p.err, MLA_DEVFLAG_TIMEOUT)))
           break;
-        mbar_arrive_expect_tx(bar(Q_FULL), nb * kQBlkBytes);
-        for (int k = 0; k < nb; ++k)
-          tma_load_3d(sbase + Lay::kOffQ + k * kQBlkBytes, &p.q_map, bar(Q_FULL), k * Lay::kCols, 0,
-                      sg.b * p.s_q + qrow);
+        mbar_arrive_expect_tx(bar(Q_FULL), nb * q_rows * 128);
+        for (int k = 0; k < nb; ++k) {
+          if (kGqa)  // rows (r, h): query row r, head h of the group
+            tma_load_3d(sbase + Lay::kOffQ + k * kQBlkBytes, &p.q_map, bar(Q_FULL), k * Lay::kCols,
+                        grp * p.hpg, sg.b * p.s_q);
+          else
+            tma_load_3d(sbase + Lay::kOffQ + k * kQBlkBytes, &p.q_map, bar(Q_FULL), k * Lay::kCols,
+                        0, sg.b * p.s_q + qrow);
+        }
         const int* bt = p.block_table + (size_t)sg.b * p.max_pages;
         for (int t = sg.t0; ok && t < sg.t1; ++t, ++g) {
           const int s = g % kStages, n = g / kStages;
@@ -187,11 +219,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
           const int y = page * p.page_size + tok % p.page_size;
           const uint32_t st = sbase + Lay::kOffKv + s * Lay::kStageBytes;
           mbar_arrive_expect_tx(bar(KV_FULL + s), (nb + nbc) * kKvBlkBytes);
-          for (int k = 0; k < nb; ++k)
-            tma_load_2d(st + k * kKvBlkBytes, &p.kv_map, bar(KV_FULL + s), k * Lay::kCols, y);
-          for (int k = 0; k < nbc; ++k)
-            tma_load_2d(st + Lay::kPvCopy + k * kKvBlkBytes, &p.kv_pv_map, bar(KV_FULL + s),
-                        k * Lay::kCols, y);
+          if (kGqa) {
+            // S operand: the group's keys, then the shared RoPE keys; the
+            // value region: the group's values
+            for (int k = 0; k < p.nbk; ++k)
+              tma_load_3d(st + k * kKvBlkBytes, &p.kv_map, bar(KV_FULL + s), k * 64, grp, y);
+            for (int k = 0; k < p.nbr; ++k)
+              tma_load_2d(st + (p.nbk + k) * kKvBlkBytes, &p.kr_map, bar(KV_FULL + s), k * 64, y);
+            for (int k = 0; k < nbc; ++k)
+              tma_load_3d(st + Lay::kPvCopy + k * kKvBlkBytes, &p.kv_map, bar(KV_FULL + s),
+                          p.d_h + k * 64, grp, y);
+          } else {
+            for (int k = 0; k < nb; ++k)
+              tma_load_2d(st + k * kKvBlkBytes, &p.kv_map, bar(KV_FULL + s), k * Lay::kCols, y);
+            for (int k = 0; k < nbc; ++k)
+              tma_load_2d(st + Lay::kPvCopy + k * kKvBlkBytes, &p.kv_pv_map, bar(KV_FULL + s),
+                          k * Lay::kCols, y);
+          }
         }
         ++seg_i;
       }
@@ -291,9 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
               // (128 bytes each) per step, 64-row blocks of 128-byte columns
               // kKvBlkBytes apart; K groups of 8 rows (bf16, 128-byte
               // swizzle) or 4 rows (tf32 copy, 32-byte atoms)
-              const uint64_t b = kTf32 ? smem_desc(st + Lay::kPvCopy + tok * 128, kKvBlkBytes, 512,
-                                                   kLayoutSW128Atom32)
-                                       : smem_desc(st + tok * 128, kKvBlkBytes, 1024, kLayoutSW128);
+              const uint64_t b =
+                  kTf32 ? smem_desc(st + Lay::kPvCopy + tok * 128, kKvBlkBytes, 512, kLayoutSW128Atom32)
+                  : kGqa ? smem_desc(st + Lay::kPvCopy + tok * 128, kKvBlkBytes, 1024, kLayoutSW128)
+                         : smem_desc(st + tok * 128, kKvBlkBytes, 1024, kLayoutSW128);
               mma(tmem + kTmemO, a, b, idPV, (j == 1 && kk == 0) ? 0u : 1u);
             }
             umma_commit(bar(KV_EMPTY + g % kStages));
@@ -313,7 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
   } else {
     // ------------------------------------------------------------ softmax
     const int q4 = warp & 3;
-    const int row = 32 * q4 + lane;  // head
+    const int row = 32 * q4 + lane;  // MMA row: head (MLA) or (query row, head of the group) (GQA)
+    const int r_row = kGqa ? row / p.hpg : qrow;                 // query row
+    const int head = kGqa ? grp * p.hpg + row % p.hpg : row;
+    const bool live = kGqa ? row < p.hpg * p.s_q : row < p.n_h;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const float c_log2 = p.scale_log2;
     ChunkWalk walk;
@@ -328,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
     };
     while (ok && walk.next(sg)) {
       const int L = p.seqlens[sg.b];
-      const int L_eff = L - p.s_q + 1 + qrow;
+      const int L_eff = L - p.s_q + 1 + r_row;
       const int n_t = sg.t1 - sg.t0;
       float m = -INFINITY, l = 0.f, l_exact = 0.f;
       for (int j = 0; j < n_t; ++j, ++g) {
@@ -433,9 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_sm100_kernel(const _
       if (!(ok = wwait(bar(PV_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1))) break;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const size_t orow = sg.whole ? (size_t)(sg.b * p.s_q + qrow) * p.n_h + row
-                                   : ((size_t)(p.split_base[sg.b] + sg.part) * p.s_q + qrow) * p.n_h + row;
-      const bool live = row < p.n_h;
+      const size_t orow = sg.whole ? (size_t)(sg.b * p.s_q + r_row) * p.n_h + head
+                                   : ((size_t)(p.split_base[sg.b] + sg.part) * p.s_q + r_row) * p.n_h + head;
       for (int c0 = 0; c0 < d_c; c0 += 32) {
         float o[32];
         tmem_ld32(tmem + lane_base + kTmemO + c0, o);
@@ -493,12 +540,15 @@ bool decode_small_sm100_supported(bool bf16, int d_c, int d_R) {
 }
 
 int decode_small_sm100_prepare() {
-  if (cudaFuncSetAttribute(decode_small_sm100_kernel<true>,
+  if (cudaFuncSetAttribute(decode_small_sm100_kernel<true, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)Layout<true>::kSmem) != cudaSuccess ||
-      cudaFuncSetAttribute(decode_small_sm100_kernel<false>,
+                           (int)Layout<true, false>::kSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(decode_small_sm100_kernel<false, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)Layout<false>::kSmem) != cudaSuccess) {
+                           (int)Layout<false, false>::kSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(decode_small_sm100_kernel<false, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Layout<false, true>::kSmem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -538,15 +588,65 @@ cudaError_t launch_decode_small_sm100(const DecodeArgs& a, const CUtensorMap& q_
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.num_chunks * a.s_q, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = a.bf16 ? Layout<false>::kSmem : Layout<true>::kSmem;
+  cfg.dynamicSmemBytes = a.bf16 ? Layout<false, false>::kSmem : Layout<true, false>::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 1 : 0;
-  return a.bf16 ? cudaLaunchKernelEx(&cfg, decode_small_sm100_kernel<false>, p)
-                : cudaLaunchKernelEx(&cfg, decode_small_sm100_kernel<true>, p);
+  return a.bf16 ? cudaLaunchKernelEx(&cfg, decode_small_sm100_kernel<false, false>, p)
+                : cudaLaunchKernelEx(&cfg, decode_small_sm100_kernel<true, false>, p);
+}
+
+cudaError_t launch_decode_gqa_sm100(const DecodeArgs& a, const GqaShape& gs, const CUtensorMap& q_map,
+                                    const CUtensorMap& kv_map, const CUtensorMap& kr_map,
+                                    cudaStream_t s) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.q_map = q_map;
+  p.kv_map = kv_map;
+  p.kr_map = kr_map;
+  p.block_table = a.block_table;
+  p.seqlens = a.seqlens;
+  p.header = a.header;
+  p.tile_prefix = a.tile_prefix;
+  p.split_base = a.split_base;
+  p.chunk_t = a.chunk_t;
+  p.chunk_b = a.chunk_b;
+  p.u = a.u;
+  p.lse = a.lse;
+  p.part_u = a.part_u;
+  p.part_lse = a.part_lse;
+  p.err = a.err;
+  p.B = a.B;
+  p.s_q = a.s_q;
+  p.n_h = a.n_h;
+  p.d_c = a.d_c;  // = d_v: the output width
+  p.max_pages = a.max_pages;
+  p.page_size = a.page_size;
+  p.num_pages = a.num_pages;
+  p.n_g = gs.n_g;
+  p.hpg = a.n_h / gs.n_g;
+  p.d_h = gs.d_h;
+  p.d_v = gs.d_v;
+  p.nbk = gs.d_h / 64;
+  p.nbr = (gs.d_R + 63) / 64;
+  p.nbv = gs.d_v / 64;
+  p.blocks = p.nbk + p.nbr;
+  p.out_f32 = a.out_f32 ? 1 : 0;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.num_chunks * gs.n_g, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<false, true>::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_small_sm100_kernel<false, true>, p);
 }
 
 }  // namespace mla

@@ -66,6 +66,17 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 // only): the cache again with 128-byte swizzle of 32-byte atoms.  Split
 // partials are fp32.
 bool decode_small_sm100_supported(bool bf16, int d_c, int d_R);
+// GQA path of GQLA on the same kernel (bf16): one CTA per (KV chunk, group),
+// every head of the group and every query row as MMA rows.  q_map: q
+// [B * s_q, n_h, d_h + d_R], box 64 x heads-per-group x s_q; kv_map: the
+// expanded cache [rows, n_g, d_h + d_v], box 64 x 1 x 64; kr_map: the RoPE
+// keys [rows, d_R], box 64 x 64; 128-byte swizzle.  a.d_c carries d_v.
+struct GqaShape {
+  int n_g, d_h, d_v, d_R;
+};
+cudaError_t launch_decode_gqa_sm100(const DecodeArgs& a, const GqaShape& gs, const CUtensorMap& q_map,
+                                    const CUtensorMap& kv_map, const CUtensorMap& kr_map,
+                                    cudaStream_t s);
 int decode_small_sm100_prepare();
 cudaError_t launch_decode_small_sm100(const DecodeArgs& a, const CUtensorMap& q_map,
                                       const CUtensorMap& kv_map, const CUtensorMap& kv_pv_map,

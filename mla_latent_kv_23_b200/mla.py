@@ -40,8 +40,21 @@ class DecodeParams(ctypes.Structure):
                 ("num_splits", ctypes.c_int), ("u_fp32", ctypes.c_int)]
 
 
+class GqaParams(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("kv", ctypes.c_void_p), ("k_rope", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("seqlens", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("s_q", ctypes.c_int), ("n_h", ctypes.c_int),
+                ("n_g", ctypes.c_int), ("d_h", ctypes.c_int), ("d_v", ctypes.c_int),
+                ("d_R", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("max_pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int),
+                ("num_splits", ctypes.c_int), ("o_fp32", ctypes.c_int)]
+
+
 _V, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _P = ctypes.POINTER(DecodeParams)
+_PG = ctypes.POINTER(GqaParams)
 SIGNATURES = {
     "mla_status_string": ([_I], ctypes.c_char_p),
     "mla_absorb_weights": ([_V, _V, _V, _I, _I, _I, _I, _I, _V], _I),
@@ -59,6 +72,8 @@ SIGNATURES = {
     "mla_decode_combine": ([_P, _V, _S, _V], _I),
     "mla_decode_kernel_info": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
     "mla_decode_noalloc": ([_P, _V], _I),
+    "mla_decode_gqa_workspace_size": ([_PG, ctypes.POINTER(_S)], _I),
+    "mla_decode_gqa": ([_PG, _V, _S, _V], _I),
     "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
     "mla_merge_partials": ([_V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
     "mla_check_device_errors": ([_V, ctypes.POINTER(_I)], _I),
@@ -348,6 +363,33 @@ def decode(q, kv_cache, block_table, seqlens, page_size: int, d_R: int, softmax_
     ws = torch.empty(max(mla_decode_workspace_size(p), 256), dtype=torch.uint8, device=q.device)
     mla_decode(p, ws, stream)
     return u, lse
+
+
+def decode_gqa(q, kv, k_rope, block_table, seqlens, page_size: int, softmax_scale: float,
+               num_splits: int = 0, o_dtype=None, with_lse: bool = True, stream=None):
+    """GQLA's GQA path: q [B, s_q, n_h, d_h + d_R], kv [rows, n_g, d_h + d_v],
+    k_rope [rows, d_R] -> (o [B, s_q, n_h, d_v], lse [B, s_q, n_h] or None)."""
+    torch = _torch()
+    B, s_q, n_h, Wq = q.shape
+    rows, n_g, Wkv = kv.shape
+    d_R = k_rope.shape[1]
+    d_h = Wq - d_R
+    d_v = Wkv - d_h
+    o = torch.empty((B, s_q, n_h, d_v), dtype=o_dtype or torch.float32, device=q.device)
+    lse = torch.empty((B, s_q, n_h), dtype=torch.float32, device=q.device) if with_lse else None
+    p = GqaParams(q=_ptr(q), kv=_ptr(kv), k_rope=_ptr(k_rope), block_table=_ptr(block_table),
+                  seqlens=_ptr(seqlens), o=_ptr(o), lse=_ptr(lse), B=B, s_q=s_q, n_h=n_h, n_g=n_g,
+                  d_h=d_h, d_v=d_v, d_R=d_R, page_size=page_size,
+                  max_pages_per_seq=block_table.shape[1], num_pages=max(rows // page_size, 1),
+                  softmax_scale=float(softmax_scale), dtype=_dtype_code(q), num_splits=num_splits,
+                  o_fp32=int(o.dtype == torch.float32))
+    n = _S(0)
+    _check(lib().mla_decode_gqa_workspace_size(ctypes.byref(p), ctypes.byref(n)),
+           "mla_decode_gqa_workspace_size")
+    ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().mla_decode_gqa(ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
+           "mla_decode_gqa")
+    return o, lse
 
 
 def default_scale(d_h: int, d_R: int) -> float:

@@ -126,7 +126,8 @@ def config(name: str, **overrides) -> Workload:
 # draws
 # ----------------------------------------------------------------------------
 _TAGS = {"seqlens": 1, "perm": 2, "cache": 3, "outlier": 4, "h_q": 5, "W_Q": 6,
-         "W_QR": 7, "W_UK": 8, "W_UV": 9, "W_DKV": 10, "W_KR": 11, "h_ctx": 12, "tail": 13}
+         "W_QR": 7, "W_UK": 8, "W_UV": 9, "W_DKV": 10, "W_KR": 11, "h_ctx": 12, "tail": 13,
+         "gqa_kv": 14, "gqa_kr": 15, "gqa_q": 16}
 
 
 _BLOCK = 1 << 22  # elements per independently seeded block of a large tensor
@@ -277,3 +278,20 @@ def random_q(w: Workload, seed_tag: int = 0) -> np.ndarray:
     q = g.standard_normal(size=(w.B, w.s_q, w.n_h, w.width), dtype=np.float32)
     q[..., :w.d_c] *= np.float32(0.5)
     return _store(q, w.dtype)
+
+
+def draw_gqa(w: Workload, n_g: int) -> dict:
+    """Inputs of a decode on GQLA's GQA path: the per-group expanded cache
+    kv [rows, n_g, d_h + d_v] (keys then values of each group, N(0, 1)), the
+    shared RoPE keys k_rope [rows, d_R] (N(0, 1), the distribution of a
+    rotated N(0, 1) vector), and q [B, s_q, n_h, d_h + d_R] (q^nope N(0, 1/4),
+    q^R N(0, 1)), with the sequence lengths and block table of ``w``."""
+    seqlens = draw_seqlens(w)
+    bt, num_pages = make_block_table(w, seqlens)
+    rows = num_pages * w.page_size
+    kv = _normal(w.seed, "gqa_kv", (rows, n_g, w.d_h + w.d_v), 1.0, w.dtype)
+    kr = _normal(w.seed, "gqa_kr", (rows, w.d_R), 1.0, w.dtype)
+    q = _normal(w.seed, "gqa_q", (w.B, w.s_q, w.n_h, w.d_h + w.d_R), 1.0, "fp32")
+    q[..., :w.d_h] *= np.float32(0.5)
+    q = _store(q, w.dtype)
+    return dict(seqlens=seqlens, block_table=bt, num_pages=num_pages, kv=kv, k_rope=kr, q=q)

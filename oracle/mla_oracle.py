@@ -313,3 +313,48 @@ def output_projection(o: np.ndarray, W_O: np.ndarray) -> np.ndarray:
 def up_project(u: np.ndarray, W_UV: np.ndarray) -> np.ndarray:
     """o_i = W^UV_i u_i: u [..., n_h, d_c], W^UV [n_h, d_v, d_c] -> [..., n_h, d_v]."""
     return np.einsum("...hc,hvc->...hv", np.asarray(u, f64), np.asarray(W_UV, f64))
+
+
+# ----------------------------------------------------------------------------
+# GQLA's GQA path (GQLA summary, abstract and method paragraphs): heads of a
+# group share W^UK_g and W^UV_g, so the cache can hold per group the expanded
+# key K^C_g = W^UK_g c and value V_g = W^UV_g c; the RoPE key stays shared.
+# ----------------------------------------------------------------------------
+def expand_gqa_cache(cache, W_UK_g, W_UV_g, d_c: int) -> tuple:
+    """Per-group expanded cache from a latent cache [rows, d_c + d_R]:
+    kv [rows, n_g, d_h + d_v] = [c W^UK_g^T || c W^UV_g^T] and the shared
+    RoPE keys [rows, d_R]."""
+    cache = np.asarray(cache, f64)
+    C, KR = cache[:, :d_c], cache[:, d_c:]
+    K = np.einsum("rc,gkc->rgk", C, np.asarray(W_UK_g, f64))
+    V = np.einsum("rc,gvc->rgv", C, np.asarray(W_UV_g, f64))
+    return np.concatenate([K, V], axis=2), KR
+
+
+def decode_gqa(q, kv, k_rope, block_table, seqlens, w, n_g: int, picks=None):
+    """GQA decode over the per-group expanded cache: head i uses group
+    g = i // (n_h / n_g); s_j = q^nope . K^C_g[j] + q^R . k^R[j] for
+    j <= L - s_q + r, a = softmax(scale s), o = sum_j a_j V_g[j].
+    Returns dict (b, r, i) -> (o [d_v], lse)."""
+    hpg = w.n_h // n_g
+    if picks is None:
+        picks = [(b, r, i) for b in range(w.B) for r in range(w.s_q) for i in range(w.n_h)]
+    out = {}
+    kv = np.asarray(kv)
+    k_rope = np.asarray(k_rope)
+    for (b, r, i) in picks:
+        L = int(seqlens[b])
+        j = np.arange(L)
+        rows = np.asarray(block_table)[b, j // w.page_size].astype(np.int64) * w.page_size + j % w.page_size
+        g = i // hpg
+        K = np.asarray(kv[rows, g, :w.d_h], f64)
+        V = np.asarray(kv[rows, g, w.d_h:], f64)
+        KR = np.asarray(k_rope[rows], f64)
+        qv = np.asarray(q[b, r, i], f64)
+        n_valid = L - w.s_q + r + 1
+        s = w.softmax_scale * (K[:n_valid] @ qv[:w.d_h] + KR[:n_valid] @ qv[w.d_h:])
+        m = s.max()
+        e = np.exp(s - m)
+        z = e.sum()
+        out[(b, r, i)] = ((e / z) @ V[:n_valid], m + math.log(z))
+    return out

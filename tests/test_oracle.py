@@ -364,3 +364,64 @@ def test_pins_catch_planted_mistakes(monkeypatch, mistake):
         orig = orc.softmax_attend
         monkeypatch.setattr(orc, "softmax_attend", lambda q, K, V, s, n_valid: orig(q, K, V, 1.0, n_valid))
     assert compare_to_brute(w, inp) > 1e-6
+
+
+# ----------------------------------------------------------------------------
+# GQLA's GQA path
+# ----------------------------------------------------------------------------
+def test_gqa_decode_brute_force():
+    w = synth.Workload(name="gqa-bf", B=2, s_q=2, n_h=4, d_model=6, d_c=8, d_h=3, d_v=2, d_R=2,
+                       page_size=2, dtype="fp32", seqlens=(3, 5), block_table="permuted", seed=13)
+    inp = synth.draw_gqa(w, n_g=2)
+    ref = orc.decode_gqa(inp["q"], inp["kv"], inp["k_rope"], inp["block_table"], inp["seqlens"], w, 2)
+    for (b, r, i), (o, lse) in ref.items():
+        g = i // 2
+        L = int(inp["seqlens"][b])
+        rid = synth.cache_row_ids(w, inp["block_table"], b, L)
+        scores = []
+        for j in range(L - w.s_q + r + 1):
+            row = rid[j]
+            dot = math.fsum([float(inp["q"][b, r, i, k]) * float(inp["kv"][row, g, k]) for k in range(w.d_h)] +
+                            [float(inp["q"][b, r, i, w.d_h + k]) * float(inp["k_rope"][row, k])
+                             for k in range(w.d_R)])
+            scores.append(w.softmax_scale * dot)
+        mx = max(scores)
+        ex = [math.exp(x - mx) for x in scores]
+        z = math.fsum(ex)
+        assert abs(lse - (mx + math.log(z))) < 1e-12
+        for v in range(w.d_v):
+            ref_v = math.fsum(ex[j] / z * float(inp["kv"][rid[j], g, w.d_h + v]) for j in range(len(ex)))
+            assert abs(o[v] - ref_v) < 1e-12
+
+
+def test_gqa_and_mla_paths_agree_with_tied_weights():
+    # the two decoding paths over the same GQLA weights: heads of a group share
+    # W^UK_g, W^UV_g; the GQA path on the expanded cache equals the MLA path
+    # (expanded definition, and absorbed u with o = W^UV_g u)
+    n_g = 2
+    w = medium_workload(s_q=2)
+    inp = synth.draw(w)
+    hpg = w.n_h // n_g
+    rng = np.random.default_rng(4)
+    W_UK_g = rng.standard_normal((n_g, w.d_h, w.d_c)) / math.sqrt(w.d_c)
+    W_UV_g = rng.standard_normal((n_g, w.d_v, w.d_c)) / math.sqrt(w.d_c)
+    tied = dict(inp)
+    tied["W_UK"] = np.repeat(W_UK_g, hpg, axis=0)
+    tied["W_UV"] = np.repeat(W_UV_g, hpg, axis=0)
+    mla_o = orc.decode_expanded(tied, w)
+    kv, kr = orc.expand_gqa_cache(inp["cache"], W_UK_g, W_UV_g, w.d_c)
+    q = np.zeros((w.B, w.s_q, w.n_h, w.d_h + w.d_R))
+    for b in range(w.B):
+        for r in range(w.s_q):
+            for i in range(w.n_h):
+                q[b, r, i] = orc.query_head(inp["W_Q"][i], inp["W_QR"][i], inp["h_q"][b, r],
+                                            int(inp["qpos"][b, r]), w.rope_base)
+    gqa = orc.decode_gqa(q, kv, kr, inp["block_table"], inp["seqlens"], w, n_g)
+    qa = np.stack([np.stack([orc.absorbed_queries(tied, w, b, r) for r in range(w.s_q)])
+                   for b in range(w.B)])
+    ua = orc.decode_absorbed(qa, inp["cache"], inp["block_table"], inp["seqlens"], w)
+    for key, (o, lse) in gqa.items():
+        o_ref, lse_ref = mla_o[key]
+        assert _max_abs(o, o_ref) < 1e-10 and abs(lse - lse_ref) < 1e-10
+        u, _ = ua[key]
+        assert _max_abs(W_UV_g[key[2] // hpg] @ u, o) < 1e-10
