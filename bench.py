@@ -225,7 +225,8 @@ def workload_config(w, l2_note):
             "B": w.B, "seq_len": int(w.seqlens[0]) if w.seqlens else None, "s_q": w.s_q,
             "n_h": w.n_h, "d_c": w.d_c, "d_R": w.d_R, "page_size": w.page_size,
             "softmax_scale": w.softmax_scale, "l2": l2_note,
-            "step": "mla_decode (plan + attend + combine) + mla_up_proj"}
+            "step": "mla_decode_step (plan + attend + combine fused into the up-projection; "
+                    "with a bf16 u: mla_decode + mla_up_proj)"}
 
 
 # ----------------------------------------------------------------------------
@@ -271,19 +272,25 @@ def run_gpu(args, w):
     lse = torch.empty((w.B, w.s_q, w.n_h), dtype=torch.float32, device=dev)
     o = torch.empty((T, w.n_h, w.d_v), dtype=tdt, device=dev)
     params = [mla.decode_params(qs[i], caches[i], bt, sl, u, lse, w.page_size, w.d_R,
-                                w.softmax_scale) for i in range(R)]
+                                w.softmax_scale, args.splits) for i in range(R)]
     ws = torch.empty(mla.mla_decode_workspace_size(params[0]), dtype=torch.uint8, device=dev)
     tc, chunks = mla.mla_decode_kernel_info(params[0])
     if not tc:
         raise RuntimeError("the tensor-core decode kernel was not selected for this workload")
 
+    fused = args.u_dtype == "fp32"
+
     def step(i, ev=None):
-        # the caller's step: mla_decode (plan, attend and combine chained by
-        # programmatic dependent launch) and the up-projection; with events,
-        # the stages are called one by one so that the attend kernel alone
-        # sits between the two event nodes
+        # the caller's step: plan, attend and (with an fp32 u) the combine
+        # fused into the up-projection, chained by programmatic dependent
+        # launch (mla_decode_step); with a bf16 u, mla_decode then
+        # mla_up_proj.  With events, the stages are called one by one so that
+        # the attend kernel alone sits between the two event nodes.
         p = params[i % R]
         if ev is None:
+            if fused:
+                mla.mla_decode_step(p, W_UV, o, ws)
+                return
             mla.mla_decode(p, ws)
         else:
             mla.mla_decode_plan(p, ws)
@@ -417,7 +424,7 @@ def run_gpu(args, w):
                 "decode_roofline_frac_step": max(t_hbm, t_tc) * 1e3 / ms_step,
                 "kv_chunks": chunks,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 4 * args.steps, "clocks": clocks}
+                "gpu_launches": (3 if fused else 4) * args.steps, "clocks": clocks}
         print(json.dumps(line), flush=True)
     graphs.clear()
     timed_graphs.clear()
@@ -446,7 +453,8 @@ def run_e2e(args, w, inp, q0, bt, sl, W_UV, dev, stream, mla, step_flops, world)
                     else tdt, device=dev)
     lse = torch.empty((w.B, w.s_q, w.n_h), dtype=torch.float32, device=dev)
     o = torch.empty((T, w.n_h, w.d_v), dtype=tdt, device=dev)
-    p = mla.decode_params(d_q, d_cache, d_bt, d_sl, u, lse, w.page_size, w.d_R, w.softmax_scale)
+    p = mla.decode_params(d_q, d_cache, d_bt, d_sl, u, lse, w.page_size, w.d_R, w.softmax_scale,
+                          args.splits)
     ws = torch.empty(mla.mla_decode_workspace_size(p), dtype=torch.uint8, device=dev)
     h2d = sum(t.numel() * t.element_size() for t in (h_cache, h_q, h_bt, h_sl))
     d2h = h_o.numel() * h_o.element_size() + h_lse.numel() * 4
@@ -456,8 +464,11 @@ def run_e2e(args, w, inp, q0, bt, sl, W_UV, dev, stream, mla, step_flops, world)
         d_q.copy_(h_q, non_blocking=True)
         d_bt.copy_(h_bt, non_blocking=True)
         d_sl.copy_(h_sl, non_blocking=True)
-        mla.mla_decode(p, ws)
-        mla.mla_up_proj(u.view(T, w.n_h, w.d_c), W_UV, o)
+        if args.u_dtype == "fp32":
+            mla.mla_decode_step(p, W_UV, o, ws)
+        else:
+            mla.mla_decode(p, ws)
+            mla.mla_up_proj(u.view(T, w.n_h, w.d_c), W_UV, o)
         h_o.copy_(o, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
 
@@ -483,7 +494,7 @@ def run_e2e(args, w, inp, q0, bt, sl, W_UV, dev, stream, mla, step_flops, world)
     mla.mla_check_device_errors(stream)
     return {"value": world * step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "steps": steps, "api": "mla_decode + mla_up_proj (C ABI via ctypes), pinned host buffers"}
+            "steps": steps, "api": "mla_decode_step (C ABI via ctypes), pinned host buffers"}
 
 
 def main():
@@ -497,6 +508,8 @@ def main():
                     help="host time for the oracle baseline (0 = skip)")
     ap.add_argument("--e2e-steps", type=int, default=20,
                     help="steps of the end-to-end (host buffers) measurement (0 = skip)")
+    ap.add_argument("--splits", type=int, default=0,
+                    help="KV chunks the batch is cut into (0: the library's automatic count)")
     ap.add_argument("--u-dtype", default="fp32", choices=["fp32", "bf16"],
                     help="type of the decode's u (fp32: the precision the parity tests hold "
                          "every workload to)")

@@ -228,6 +228,23 @@ mla_status mla_decode_combine(const mla_decode_params* p, void* workspace,
                               size_t workspace_bytes, void* stream);
 
 /*
+ * One decode step of the attention output: mla_decode, then o = W_UV u
+ * (as mla_up_proj), with the combine of split rows done inside the
+ * up-projection: each up-projection CTA merges the fp32 partials of its
+ * head's rows from the workspace (also writing u and lse), splits the fp32
+ * rows into two bf16 terms and runs the tensor-core product.  The three
+ * kernels (plan, attend, merge + up-projection) are chained by programmatic
+ * dependent launch, so the weight read starts while the attend kernel ends.
+ * Requires the DeepSeek-V3 shape kernel (bf16, d_c = 512, d_R = 64), an fp32
+ * u (p->u_fp32 = 1) and d_v <= 128.  Results equal mla_decode followed by
+ * mla_up_proj.  The workspace is mla_decode's.
+ *   W_UV  [n_h, d_v, d_c] bf16 device, read
+ *   o     [B * s_q, n_h, d_v] bf16 device, written
+ */
+mla_status mla_decode_step(const mla_decode_params* p, const void* W_UV, void* o, int d_v,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * mla_decode without a caller-provided workspace.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate
  * device memory, such as a host framework that owns all device memory and

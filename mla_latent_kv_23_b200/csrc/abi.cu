@@ -426,10 +426,40 @@ mla_status mla_decode(const mla_decode_params* p, void* ws, size_t ws_bytes, voi
   mla_status st = resolve(p, ws, ws_bytes, &r);
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
+  // the DeepSeek-V3 shape kernel plans its own chunk
+  if (r.kernel != Kernel::kV3 && (st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
   if ((st = attend(r, p, s, true)) != MLA_OK) return st;
   r.a.pdl = true;
   return cuda_status(launch_combine(r.a, s));
+}
+
+mla_status mla_decode_step(const mla_decode_params* p, const void* W_UV, void* o, int d_v,
+                           void* ws, size_t ws_bytes, void* stream) {
+  if (p != nullptr && p->B == 0) return validate_decode(p);
+  if (W_UV == nullptr || o == nullptr || d_v < 1) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W_UV) || !aligned16(o)) return MLA_ERR_INVALID_ARG;
+  Resolved r;
+  mla_status st = resolve(p, ws, ws_bytes, &r);
+  if (st != MLA_OK) return st;
+  if (r.kernel != Kernel::kV3 || !r.a.out_f32 || d_v > 128 || !r.dev->up_proj_tc)
+    return MLA_ERR_UNSUPPORTED;
+  if ((long long)p->n_h * d_v > INT_MAX) return MLA_ERR_UNSUPPORTED;
+  CUtensorMap w_map;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)p->d_c, (cuuint64_t)p->n_h * d_v};
+    const cuuint64_t strides[1] = {(cuuint64_t)p->d_c * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    if (g_encode(&w_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W_UV), dims, strides,
+                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = attend(r, p, s, true)) != MLA_OK) return st;  // plans its own chunk
+  const int T = p->B * p->s_q;
+  return cuda_status(launch_up_proj_sm100_f32u(w_map, static_cast<const float*>(p->u), o, r.dev->flags, T,
+                                               p->n_h, p->d_c, d_v, true, s, &r.a));
 }
 
 mla_status mla_absorb_weights(const void* W_UK, const void* W_Q, void* W_QK, int n_h, int d_h,

@@ -139,9 +139,13 @@ cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_
                                  int* err, int T, int n_h, int d_c, int d_v, bool f32, bool pdl,
                                  cudaStream_t s);
 // bf16 W and o with an fp32 u, read with plain loads and split into two bf16
-// terms, u = hi + lo, in shared memory: o = W^UV hi + W^UV lo.
+// terms, u = hi + lo, in shared memory: o = W^UV hi + W^UV lo.  With
+// `merge` (d_c = 512), the rows of split sequences are first merged from the
+// decode workspace's fp32 partials (and written to u and lse): the combine
+// stage fused into the up-projection.
 cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, void* o, int* err,
-                                      int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s);
+                                      int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s,
+                                      const DecodeArgs* merge = nullptr);
 
 // Weight-streaming projection Y[m, t] = sum_k W[m, k] X[t, k] on the tensor
 // cores (bf16): one CTA per (128-row tile, K slice), fp32 split-K

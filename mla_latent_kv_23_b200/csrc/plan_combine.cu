@@ -239,9 +239,10 @@ __global__ void __launch_bounds__(kCombineThreads)
   constexpr int kVecs = kPartBf16 ? 2 : 4;  // 16-byte loads per lane per partial row
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
-  // The plan stage's outputs are read before waiting: that stage completed
-  // before the attend stage that precedes this one passed its own wait, and
-  // this kernel starts only after the attend stage has passed it.
+  // The tile prefix and split bases come from the plan stage or from the
+  // attend stage itself: read them after the wait.
+  ptx::pdl_wait_previous();
+  ptx::pdl_launch_dependents();
   int sb0 = 0, sb1 = 0, tp0 = 0, tp1 = 0;
   int h = 0, br = 0, r = 0;
   if (row < rows) {
@@ -254,8 +255,6 @@ __global__ void __launch_bounds__(kCombineThreads)
     tp0 = tile_prefix[b];
     tp1 = tile_prefix[b + 1];
   }
-  ptx::pdl_wait_previous();
-  ptx::pdl_launch_dependents();
   if (row >= rows) return;
   const int nsplit = sb1 - sb0;
   if (nsplit == 0 && tp1 != tp0) return;  // written directly by the attend stage

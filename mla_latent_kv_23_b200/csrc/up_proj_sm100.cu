@@ -18,6 +18,12 @@
 // whole cost of this step) is issued before the kernel waits for the
 // previous kernel, so under programmatic dependent launch it overlaps the
 // end of the decode that produces u.
+//
+// kSplitU can also merge the split-KV partial results itself (the combine
+// of mla_decode, fused in): a row whose sequence was cut into pieces gets
+// lse = log sum_s exp(lse_s) and u = sum_s exp(lse_s - lse) u_s from the fp32
+// partials (written to u and lse as well), a whole row is read as the attend
+// stage wrote it; either way the fp32 row then enters the MMA as hi + lo.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -49,6 +55,14 @@ struct Params {
   CUtensorMap w_map;   // W_UV as [n_h * d_v rows, d_c cols], box (128 bytes) x 128 rows
   CUtensorMap u_map;   // u as [T, n_h, d_c], box (128 bytes) x 1 x n_pad (kBf16, kTf32)
   const float* u_f32;  // u (kSplitU)
+  // kSplitU with merge: the decode workspace's plan and partials (d_c = 512)
+  int merge, s_q;
+  const int* tile_prefix;
+  const int* split_base;
+  const float* part_u;
+  const float* part_lse;
+  float* u_out;        // = u_f32: merged rows are written back
+  float* lse_out;      // may be null
   void* o;             // [T, n_h, d_v]: bf16 (kBf16, kSplitU) or fp32 (kTf32)
   int* err;
   int T, n_h, d_c, d_v, n_pad;
@@ -97,6 +111,106 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
   pdl_wait_previous();
   pdl_launch_dependents();
   if constexpr (kMode == UpMode::kSplitU) {
+   if (p.merge) {
+    // one warp per row t; lane l owns columns [16 l, 16 l + 16) of d_c = 512
+    for (int tt = warp; tt < p.n_pad; tt += kThreads / 32) {
+      const int t = t0 + tt;
+      float acc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+      if (t < p.T) {
+        const int b = t / p.s_q, r = t % p.s_q;
+        const int sb0 = p.split_base[b], nsplit = p.split_base[b + 1] - sb0;
+        const size_t urow = (size_t)t * p.n_h + head;
+        float* up = p.u_out + urow * 512 + 16 * lane;
+        if (nsplit == 0) {
+          if (p.tile_prefix[b + 1] != p.tile_prefix[b]) {  // written whole by the attend stage
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 v = reinterpret_cast<const float4*>(up)[i];
+              acc[4 * i] = v.x; acc[4 * i + 1] = v.y; acc[4 * i + 2] = v.z; acc[4 * i + 3] = v.w;
+            }
+          } else {  // no tokens (a rejected length): u = 0, lse = -inf
+#pragma unroll
+            for (int i = 0; i < 4; ++i) reinterpret_cast<float4*>(up)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lane == 0 && p.lse_out) p.lse_out[urow] = -INFINITY;
+          }
+        } else {
+          const size_t slot0 = (size_t)sb0 * p.s_q + r;  // slot of split s: slot0 + s s_q
+          auto lse_of = [&](int sp) { return p.part_lse[(slot0 + (size_t)sp * p.s_q) * p.n_h + head]; };
+          float m = -INFINITY, z = 0.f;
+          for (int sp = lane; sp < nsplit; sp += 32) {
+            const float x = lse_of(sp);
+            if (x > m) {
+              z = z * expf(m - x) + 1.f;
+              m = x;
+            } else if (x != -INFINITY) {
+              z += expf(x - m);
+            }
+          }
+          float m_all = m;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m_all = fmaxf(m_all, __shfl_xor_sync(0xffffffffu, m_all, o));
+          z = m == -INFINITY ? 0.f : z * expf(m - m_all);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+          const float lse = m_all == -INFINITY ? -INFINITY : m_all + logf(z);
+          if (m_all != -INFINITY) {
+            for (int s0 = 0; s0 < nsplit; s0 += 4) {
+              float4 v[4][4];
+              const int n_here = min(4, nsplit - s0);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (k < n_here) {
+                  const float4* src = reinterpret_cast<const float4*>(
+                      p.part_u + ((slot0 + (size_t)(s0 + k) * p.s_q) * p.n_h + head) * 512 + 16 * lane);
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) v[k][i] = src[i];
+                }
+              const float w_me = lane < n_here ? expf(lse_of(s0 + lane) - lse) : 0.f;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float w = __shfl_sync(0xffffffffu, w_me, k);
+                if (k < n_here) {
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    acc[4 * i] += w * v[k][i].x;
+                    acc[4 * i + 1] += w * v[k][i].y;
+                    acc[4 * i + 2] += w * v[k][i].z;
+                    acc[4 * i + 3] += w * v[k][i].w;
+                  }
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<float4*>(up)[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+          if (lane == 0 && p.lse_out) p.lse_out[urow] = lse;
+        }
+      }
+      // the row's two bf16 terms: lane l's 16 columns are chunks 2l, 2l + 1
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float a0 = acc[8 * c + 2 * k], a1 = acc[8 * c + 2 * k + 1];
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+          const float2 hf = __bfloat1622float2(h2);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+          hi[k] = *reinterpret_cast<const uint32_t*>(&h2);
+          lo[k] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
+        const int c8 = 2 * lane + c, kb = c8 >> 3, k16 = c8 & 7;
+        const uint32_t off = kb * ublk + tt * 128 + ((static_cast<uint32_t>(k16 ^ (tt & 7))) << 4);
+        st_shared_v4(sbase + off_u + off, hi[0], hi[1], hi[2], hi[3]);
+        st_shared_v4(sbase + off_u + kMaxKb * ublk + off, lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+   } else {
     // u rows -> hi and lo bf16 terms, 8 columns (one 16-byte chunk of each
     // term) per step, in the 128-byte swizzle the MMA descriptor expects:
     // chunk k of row t at byte t * 128 + ((k ^ (t & 7)) << 4) of its block;
@@ -131,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
     }
     fence_proxy_async_smem();
     __syncthreads();
+   }
   }
   bool ok = true;
   if (threadIdx.x == 0) {
@@ -252,9 +367,21 @@ cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_
 }
 
 cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, void* o, int* err,
-                                      int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s) {
+                                      int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s,
+                                      const DecodeArgs* merge) {
   Params p;
+  memset(&p, 0, sizeof(p));
   p.w_map = w_map;
+  if (merge != nullptr) {
+    p.merge = 1;
+    p.s_q = merge->s_q;
+    p.tile_prefix = merge->tile_prefix;
+    p.split_base = merge->split_base;
+    p.part_u = merge->part_u;
+    p.part_lse = merge->part_lse;
+    p.u_out = const_cast<float*>(u);
+    p.lse_out = merge->lse;
+  }
   memset(&p.u_map, 0, sizeof(p.u_map));
   p.u_f32 = u;
   p.o = o;

@@ -72,6 +72,7 @@ SIGNATURES = {
     "mla_decode_combine": ([_P, _V, _S, _V], _I),
     "mla_decode_kernel_info": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
     "mla_decode_noalloc": ([_P, _V], _I),
+    "mla_decode_step": ([_P, _V, _V, _I, _V, _S, _V], _I),
     "mla_decode_gqa_workspace_size": ([_PG, ctypes.POINTER(_S)], _I),
     "mla_decode_gqa": ([_PG, _V, _S, _V], _I),
     "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
@@ -294,6 +295,15 @@ def mla_decode_attend(p: DecodeParams, workspace, stream=None) -> None:
 
 def mla_decode_combine(p: DecodeParams, workspace, stream=None) -> None:
     _stage("mla_decode_combine", p, workspace, stream)
+
+
+def mla_decode_step(p: DecodeParams, W_UV, o, workspace, stream=None) -> None:
+    """mla_decode then o = W_UV u with the combine fused into the
+    up-projection (fp32 u, the DeepSeek-V3 shape): o [B * s_q, n_h, d_v]."""
+    d_v = W_UV.shape[1]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().mla_decode_step(ctypes.byref(p), _ptr(W_UV), _ptr(o), d_v, _ptr(workspace), nbytes,
+                                 _stream(stream)), "mla_decode_step")
 
 
 def mla_decode_noalloc(p: DecodeParams, stream=None) -> None:

@@ -385,3 +385,30 @@ def test_merge_partials_against_its_definition(dtype, d_c, R):
     tol = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
     err = (got_u[fin] - u_ref[fin]).abs() / (1 + u_ref[fin].abs())
     assert err.max() <= tol
+
+
+@pytest.mark.parametrize("s_q,splits", [(1, 0), (1, 5), (2, 0), (2, 3)])
+def test_decode_step_fuses_the_combine_into_the_up_projection(s_q, splits):
+    # mla_decode_step merges split rows inside the up-projection; it returns
+    # what mla_decode followed by mla_up_proj returns, bit for bit (the same
+    # arithmetic in the same order), and meets the oracle's bounds
+    w = v3_small(s_q=s_q, B=5, seqlens=(100, 1000, 777, 64, 2))
+    inp = synth.draw(w)
+    q = synth.random_q(w)
+    qd, cache = to_dev(q, w), to_dev(inp["cache"], w)
+    bt, sl = to_dev_i32(inp["block_table"]), to_dev_i32(inp["seqlens"])
+    W_UV = to_dev(inp["W_UV"], w)
+    T = w.B * w.s_q
+    u1, l1 = mla.decode(qd, cache, bt, sl, w.page_size, w.d_R, w.softmax_scale, splits)
+    o1 = torch.empty((T, w.n_h, w.d_v), dtype=torch.bfloat16, device="cuda")
+    mla.mla_up_proj(u1.view(T, w.n_h, w.d_c), W_UV, o1)
+    u2, l2 = torch.full_like(u1, float("nan")), torch.full_like(l1, float("nan"))
+    o2 = torch.full_like(o1, float("nan"))
+    p = mla.decode_params(qd, cache, bt, sl, u2, l2, w.page_size, w.d_R, w.softmax_scale, splits)
+    ws = torch.empty(mla.mla_decode_workspace_size(p), dtype=torch.uint8, device="cuda")
+    mla.mla_decode_step(p, W_UV, o2, ws)
+    mla.mla_check_device_errors()
+    assert torch.equal(u1, u2) and torch.equal(l1, l2) and torch.equal(o1, o2)
+    out = dict(u=u2, lse=l2, o=o2.view(w.B, w.s_q, w.n_h, w.d_v))
+    picks = [(b, r, i) for b in range(w.B) for r in range(s_q) for i in (0, 1, 64, 127)]
+    assert_tight(check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"]))
