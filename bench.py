@@ -424,7 +424,7 @@ def run_gpu(args, w):
                 "decode_roofline_frac_step": max(t_hbm, t_tc) * 1e3 / ms_step,
                 "kv_chunks": chunks,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": (3 if fused else 4) * args.steps, "clocks": clocks}
+                "gpu_launches": (3 if fused else 4) * (args.steps - n_ev) + 4 * n_ev, "clocks": clocks}
         print(json.dumps(line), flush=True)
     graphs.clear()
     timed_graphs.clear()

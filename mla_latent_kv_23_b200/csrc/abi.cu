@@ -243,6 +243,40 @@ mla_status run_projection(WgemmLaunch L, const void* X, int K, int T, int ldx_ro
   return MLA_OK;
 }
 
+// 4D map over the cache [rows, 576] (bf16) that gathers one CTA's latent
+// half of 64 rows in one copy: dimensions (column, row, block & 1,
+// block >> 1) with byte strides (1152, 128, 512) and box 64 x 64 x 2 x 2, so
+// that the copy at column 128 r holds the blocks starting at columns
+// 128 r + {0, 64, 256, 320}, block k at k x 8 KB (rows of 128 bytes, 128-byte
+// swizzle).  Every address stays inside the row (column <= 511).
+bool encode_kv_lat4(CUtensorMap* m, const void* ptr, uint64_t rows) {
+  const cuuint64_t dims[4] = {192, rows, 2, 2};
+  const cuuint64_t strides[3] = {576 * 2, 128, 512};
+  const cuuint32_t box[4] = {64, 64, 2, 2};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 5D map over the queries [B * s_q, n_h, 576] (bf16, n_h % 16 == 0) that
+// fills one CTA's query area in one copy per 64-column block: dimensions
+// (column, head within 16, column half, group of 16 heads, query row), the
+// column half's stride 128 columns (latent) or 32 (RoPE), box box_x x 16 x 2
+// x 4 x 1, so that shared row 32 g + 16 j + i holds head 16 g + i at the
+// columns of half j.  Latent copies start at columns {0, 64, 256, 320} and
+// the RoPE copy at 512: every address stays inside the head's row.
+bool encode_q5(CUtensorMap* m, const void* ptr, uint64_t n_h, uint64_t qrows, bool rope) {
+  const cuuint64_t dims[5] = {rope ? 544u : 384u, 16, 2, n_h / 16, qrows};
+  const cuuint64_t strides[4] = {576 * 2, rope ? 64u : 256u, 16 * 576 * 2, n_h * 576 * 2};
+  const cuuint32_t box[5] = {rope ? 32u : 64u, 16, 2, 4, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  rope ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3D map over the queries [B * s_q, n_h, 576] (bf16), box box_x x 16 heads x 1.
 mla_status encode_q(CUtensorMap* m, const void* ptr, uint64_t n_h, uint64_t qrows, uint32_t box_x,
                     CUtensorMapSwizzle sw) {
@@ -322,6 +356,9 @@ mla_status attend(Resolved r, const mla_decode_params* p, cudaStream_t s, bool p
   if ((st = encode_q(&maps.q_lat, p->q, p->n_h, qrows, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
       (st = encode_q(&maps.q_rope, p->q, p->n_h, qrows, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
     return st;
+  maps.has_kv4 = encode_kv_lat4(&maps.kv_lat4, p->kv_cache, kvrows) ? 1 : 0;
+  maps.has_q5 = p->n_h % 16 == 0 && encode_q5(&maps.q_lat5, p->q, p->n_h, qrows, false) &&
+                encode_q5(&maps.q_rope5, p->q, p->n_h, qrows, true);
   if ((st = encode_out(&maps.u_out, p->u, p->n_h, qrows, r.a.out_f32)) != MLA_OK ||
       (st = encode_out(&maps.part_out, r.a.part_u, p->n_h, (uint64_t)r.slots, r.a.out_f32)) !=
           MLA_OK)
@@ -426,8 +463,7 @@ mla_status mla_decode(const mla_decode_params* p, void* ws, size_t ws_bytes, voi
   mla_status st = resolve(p, ws, ws_bytes, &r);
   if (st != MLA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the DeepSeek-V3 shape kernel plans its own chunk
-  if (r.kernel != Kernel::kV3 && (st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
+  if ((st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
   if ((st = attend(r, p, s, true)) != MLA_OK) return st;
   r.a.pdl = true;
   return cuda_status(launch_combine(r.a, s));
@@ -456,7 +492,8 @@ mla_status mla_decode_step(const mla_decode_params* p, const void* W_UV, void* o
       return MLA_ERR_CUDA;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = attend(r, p, s, true)) != MLA_OK) return st;  // plans its own chunk
+  if ((st = cuda_status(launch_plan(r.a, s))) != MLA_OK) return st;
+  if ((st = attend(r, p, s, true)) != MLA_OK) return st;
   const int T = p->B * p->s_q;
   return cuda_status(launch_up_proj_sm100_f32u(w_map, static_cast<const float*>(p->u), o, r.dev->flags, T,
                                                p->n_h, p->d_c, d_v, true, s, &r.a));

@@ -93,8 +93,7 @@ constexpr uint32_t kOffP = kOffKv + kStages * kStageBytes;   // [2] second halve
 constexpr uint32_t kOffMax = kOffP + 2 * kPHalf;             // float [2 tile parity][64 heads]
 constexpr uint32_t kOffSum = kOffMax + 2 * 64 * 4;           // float [2 kind][2 group][64 heads]
 constexpr uint32_t kOffScratch = kOffSum + 2 * 2 * 64 * 4;    // 16 words written by the odd CTA's signals
-constexpr uint32_t kOffPlan = kOffScratch + 64;               // this chunk's ChunkStart
-constexpr uint32_t kOffBar = kOffPlan + 64;
+constexpr uint32_t kOffBar = kOffScratch + 64;
 
 // Barriers of the even CTA that the odd CTA signals ("paired" below) count
 // the even CTA's own arrivals, and the odd CTA's signals as 4-byte
@@ -145,14 +144,14 @@ struct Params {
   const int* block_table;
   const int* seqlens;
   const int* header;
-  const int* tile_prefix;  // written by CTA 0 (the merge of partial rows reads it)
+  const int* tile_prefix;
   const int* split_base;
   const int* chunk_t;
   const int* chunk_b;
   float* part_lse;
   float* lse;
   int* err;
-  int B, s_q, n_h, max_pages, page_size, num_pages, num_chunks;
+  int B, s_q, n_h, max_pages, page_size, num_pages;
   int out_f32;       // u and the split partials are fp32 (else bf16)
   float scale_log2;  // softmax_scale * log2(e)
 };
@@ -242,40 +241,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_relinquish_pair();
   }
   if (warp == kWarpTma && lane == 0) {
-    prefetch_tmap(&p.maps.kv_lat);
+    prefetch_tmap(p.maps.has_kv4 ? &p.maps.kv_lat4 : &p.maps.kv_lat);
     prefetch_tmap(&p.maps.kv_rope);
   }
   if (warp == kWarpRelay && lane == 0) {
-    prefetch_tmap(&p.maps.q_lat);
-    prefetch_tmap(&p.maps.q_rope);
+    prefetch_tmap(p.maps.has_q5 ? &p.maps.q_lat5 : &p.maps.q_lat);
+    prefetch_tmap(p.maps.has_q5 ? &p.maps.q_rope5 : &p.maps.q_rope);
   }
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // both CTAs' barriers and TMEM exist before either uses the other's
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base + kOffTmemSlot);
-  // everything above overlaps the previous kernel; inputs are read below
+  // everything above overlaps the plan kernel; its results are read below
   pdl_wait_previous();
   pdl_launch_dependents();
-  // The chunk's place on the cost line, computed here from the sequence
-  // lengths (the plan stage's cut); CTA 0 also writes the tile prefix and the
-  // split bases that the merge of partial rows reads.
-  if (warp == kWarpRelay) {
-    const bool first = blockIdx.x == 0;
-    const ChunkStart cs0 =
-        plan_chunk(p.seqlens, p.B, p.s_q, p.max_pages * p.page_size, p.num_chunks, chunk,
-                   first ? const_cast<int*>(p.tile_prefix) : nullptr,
-                   first ? const_cast<int*>(p.split_base) : nullptr, first ? p.err : nullptr);
-    if (lane == 0) *reinterpret_cast<ChunkStart*>(base + kOffPlan) = cs0;
-  }
-  __syncthreads();
-  const ChunkStart cs = *reinterpret_cast<const ChunkStart*>(base + kOffPlan);
-  const int max_len = p.max_pages * p.page_size;
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ producer
-    SeqWalk walk;
-    walk.init(cs, p.seqlens, p.B, p.s_q, max_len, chunk);
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
     Segment sg;
     int g = 0;
     int last_n[kStages], tail_n[kStages];  // uses of LOCAL_FULL per stage
@@ -326,23 +311,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // tail tile: this CTA's relay zeroes the rows past the end
                 // once they land, then signals the even CTA
                 mbar_arrive_expect_tx(bar(LOCAL_FULL + s), kStageBytes);
-                for (int kc = 0; kc < 4; ++kc)
-                  tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(LOCAL_FULL + s),
-                              lat_col(kc, (int)rank), y);
+                if (p.maps.has_kv4)
+                  tma_load_4d(st, &p.maps.kv_lat4, bar(LOCAL_FULL + s), 128 * (int)rank, y, 0, 0);
+                else
+                  for (int kc = 0; kc < 4; ++kc)
+                    tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(LOCAL_FULL + s),
+                                lat_col(kc, (int)rank), y);
                 tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(LOCAL_FULL + s),
                             kDc + 32 * (int)rank, y);
                 last_n[s] = tail_n[s]++;
               } else if (leader) {
                 // full tile: both CTAs' bytes complete on the even CTA's barrier
                 mbar_arrive_expect_tx(bar(KV_FULL + s), 2 * kStageBytes);
-                for (int kc = 0; kc < 4; ++kc)
-                  tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
-                              lat_col(kc, 0), y);
+                if (p.maps.has_kv4)
+                  tma_load_4d(st, &p.maps.kv_lat4, bar(KV_FULL + s), 0, y, 0, 0);
+                else
+                  for (int kc = 0; kc < 4; ++kc)
+                    tma_load_2d(st + kc * kKvBlk, &p.maps.kv_lat, bar(KV_FULL + s),
+                                lat_col(kc, 0), y);
                 tma_load_2d(st + 4 * kKvBlk, &p.maps.kv_rope, bar(KV_FULL + s), kDc, y);
               } else {
                 const uint32_t full = mapa(bar(KV_FULL + s), 0);
-                for (int kc = 0; kc < 4; ++kc)
-                  tma_load_2d_to_pair(st + kc * kKvBlk, &p.maps.kv_lat, full, lat_col(kc, 1), y);
+                if (p.maps.has_kv4)
+                  tma_load_4d_to_pair(st, &p.maps.kv_lat4, full, 128, y, 0, 0);
+                else
+                  for (int kc = 0; kc < 4; ++kc)
+                    tma_load_2d_to_pair(st + kc * kKvBlk, &p.maps.kv_lat, full, lat_col(kc, 1), y);
                 tma_load_2d_to_pair(st + 4 * kKvBlk, &p.maps.kv_rope, full, kDc + 32, y);
               }
             }
@@ -361,8 +355,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kWarpRelay) {
     // ------------------------------------------------------------ relay
-    SeqWalk walk;
-    walk.init(cs, p.seqlens, p.B, p.s_q, max_len, chunk);
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
     Segment sg;
     int g = 0, seg_i = 0;
     int tail_n[kStages];  // uses of LOCAL_FULL per stage, in tile order
@@ -381,22 +375,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const int z = sg.b * p.s_q + qrow;
         mbar_arrive_expect_tx(bar(Q_LOCAL), kQBytes);
-        for (int qd = 0; qd < 4; ++qd)
-          for (int j = 0; j < 2; ++j) {
-            const int y = 64 * (int)rank + 16 * qd;
-            const uint32_t r0 = static_cast<uint32_t>(32 * qd + 16 * j);
-            for (int kc = 0; kc < 4; ++kc)
-              tma_load_3d(sbase + kOffQ + kc * kQBlk + r0 * 128, &p.maps.q_lat, bar(Q_LOCAL),
-                          lat_col(kc, j), y, z);
-            tma_load_3d(sbase + kOffQ + 4 * kQBlk + r0 * 64, &p.maps.q_rope, bar(Q_LOCAL),
-                        kDc + 32 * j, y, z);
-          }
+        if (p.maps.has_q5) {
+          // one copy per 64-column block: rows 32 qd + 16 j + i at once
+          for (int kc = 0; kc < 4; ++kc)
+            tma_load_5d(sbase + kOffQ + kc * kQBlk, &p.maps.q_lat5, bar(Q_LOCAL), lat_col(kc, 0),
+                        0, 0, 4 * (int)rank, z);
+          tma_load_5d(sbase + kOffQ + 4 * kQBlk, &p.maps.q_rope5, bar(Q_LOCAL), kDc, 0, 0,
+                      4 * (int)rank, z);
+        } else {
+          for (int qd = 0; qd < 4; ++qd)
+            for (int j = 0; j < 2; ++j) {
+              const int y = 64 * (int)rank + 16 * qd;
+              const uint32_t r0 = static_cast<uint32_t>(32 * qd + 16 * j);
+              for (int kc = 0; kc < 4; ++kc)
+                tma_load_3d(sbase + kOffQ + kc * kQBlk + r0 * 128, &p.maps.q_lat, bar(Q_LOCAL),
+                            lat_col(kc, j), y, z);
+              tma_load_3d(sbase + kOffQ + 4 * kQBlk + r0 * 64, &p.maps.q_rope, bar(Q_LOCAL),
+                          kDc + 32 * j, y, z);
+            }
+        }
       }
       q_in_flight = true;
       // the next segment's query rows go to L2 now, so that its TMA load
       // after this segment's last S is an L2 hit
       if (lane == 0) {
-        SeqWalk peek = walk;
+        ChunkWalk peek = walk;
         Segment nx;
         const int heads = min(64, p.n_h - 64 * (int)rank);
         if (heads > 0 && peek.next(nx)) {
@@ -450,8 +453,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (leader) {
       constexpr uint32_t kIdS = idesc_bf16(256, 128, false);
       constexpr uint32_t kIdPV = idesc_bf16(128, 256, true);
-      SeqWalk walk;
-      walk.init(cs, p.seqlens, p.B, p.s_q, max_len, chunk);
+      ChunkWalk walk;
+      walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
       Segment sg;
       int g0 = 0, seg_i = 0;
       bool ok = true;
@@ -570,8 +573,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       return live && warp_wait(bar(GRP), ph, p.err);
     };
 
-    SeqWalk walk;
-    walk.init(cs, p.seqlens, p.B, p.s_q, max_len, chunk);
+    ChunkWalk walk;
+    walk.init(p.tile_prefix, p.chunk_t, p.chunk_b, p.header, p.B, chunk);
     Segment sg;
     int g = 0;
     bool ok = true;
@@ -583,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // the segment's output row: u's row, or its partial slot (read now,
       // used by the epilogue)
       const int out_z =
-          sg.whole ? sg.b * p.s_q + qrow : (sg.split_base + sg.part) * p.s_q + qrow;
+          sg.whole ? sg.b * p.s_q + qrow : (p.split_base[sg.b] + sg.part) * p.s_q + qrow;
       // this group's sums over its own tiles of the segment, in the scale of
       // m_used (the maximum it last applied)
       float m_used = -INFINITY, l = 0.f, l_exact = 0.f;
@@ -904,7 +907,6 @@ cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cuda
   p.max_pages = a.max_pages;
   p.page_size = a.page_size;
   p.num_pages = a.num_pages;
-  p.num_chunks = a.num_chunks;
   p.out_f32 = a.out_f32 ? 1 : 0;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   cudaLaunchConfig_t cfg = {};

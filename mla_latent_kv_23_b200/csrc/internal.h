@@ -92,8 +92,18 @@ cudaError_t launch_decode_small_sm100(const DecodeArgs& a, const CUtensorMap& q_
 // [slots, n_h, 512], both bf16 (boxes 64 x 32 heads x 1) or both fp32
 // (boxes 32 x 32 heads x 1), 128-byte swizzle, for the TMA stores of the
 // epilogue; heads past n_h are not written.
+//
+// kv_lat4 covers one CTA's four 64-column latent blocks of 64 rows in one
+// copy: dimensions (column, row, block & 1, block >> 1) with byte strides
+// (1152, 128, 512); q_lat5 / q_rope5 cover a CTA's whole query area in one
+// copy each: (column, head within 16, column half, group of 16 heads, query
+// row) with the column half's stride 256 / 64 bytes.  has_kv4 / has_q5 say
+// whether they were encoded (has_q5 needs n_h % 16 == 0); otherwise the
+// kernel issues the per-block copies.
 struct Sm100Maps {
   CUtensorMap kv_lat, kv_rope, q_lat, q_rope, u_out, part_out;
+  CUtensorMap kv_lat4, q_lat5, q_rope5;
+  int has_kv4, has_q5;
 };
 cudaError_t launch_decode_sm100(const DecodeArgs& a, const Sm100Maps& maps, cudaStream_t s);
 size_t decode_sm100_smem_bytes();
