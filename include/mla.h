@@ -371,6 +371,18 @@ mla_status mla_output_projection(const void* x, mla_dtype x_dtype, const void* W
 mla_status mla_merge_partials(const void* u_parts, const float* lse_parts, void* u, float* lse,
                               int R, int rows, int d_c, mla_dtype dtype, void* stream);
 
+/*
+ * Self-test of the bounded device-side wait.  Launches one kernel that
+ * waits on an mbarrier phase with a limit of about 2e6 cycles (~1 ms):
+ * with arrive != 0 the kernel first completes that phase and the wait
+ * returns at once; with arrive == 0 nothing completes it, the wait gives up,
+ * MLA_DEVFLAG_TIMEOUT is set in the device flags and the kernel returns.
+ * Every kernel of the library waits this way (with a limit of 2e9 cycles),
+ * so a broken hand-off ends as a flag, never as a hang.  Read the flags with
+ * mla_check_device_errors.  No arithmetic of the method is involved.
+ */
+mla_status mla_selftest_wait(int arrive, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device flag of the
  * current device.  Returns MLA_OK if no flag was raised, otherwise
  * MLA_ERR_DEVICE_CHECK and the MLA_DEVFLAG_* bits in *flags (may be NULL). */

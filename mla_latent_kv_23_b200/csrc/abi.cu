@@ -385,7 +385,7 @@ WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks) {
   L.chunk_t = off;
   off = align_up(off + sizeof(int) * (num_chunks + 1), 256);
   L.chunk_b = off;
-  off = align_up(off + sizeof(int) * num_chunks, 256);
+  off = align_up(off + sizeof(int) * 2 * (size_t)num_chunks, 256);
   L.part_lse = off;
   off = align_up(off + sizeof(float) * (size_t)L.slots * n_h, 256);
   L.part_u = off;
@@ -1007,6 +1007,13 @@ mla_status mla_merge_partials(const void* u_parts, const float* lse_parts, void*
   if (st != MLA_OK) return st;
   return cuda_status(launch_merge(u_parts, lse_parts, u, lse, R, rows, d_c,
                                   dtype == MLA_DTYPE_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_selftest_wait(int arrive, void* stream) {
+  const DeviceInfo* d = nullptr;
+  mla_status st = device_info(&d);
+  if (st != MLA_OK) return st;
+  return cuda_status(launch_wait_selftest(d->flags, arrive != 0, static_cast<cudaStream_t>(stream)));
 }
 
 mla_status mla_check_device_errors(void* stream, int* flags) {

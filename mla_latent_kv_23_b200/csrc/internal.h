@@ -22,8 +22,11 @@ constexpr int kSegCostTiles = 4;
 
 // Workspace of mla_decode.  Header ints: [0] total tiles, [1] line units per
 // chunk, [2] number of chunks, [3] split rows in use, [4] units per sequence
-// start.  chunk_t[c] is the first tile of chunk c (chunk_t[chunks] = total
-// tiles), chunk_b[c] the sequence that tile belongs to.
+// start, [5] 1 when the chunks follow the sequences (see the plan kernel).
+// chunk_t[c] is the first tile of chunk c (chunk_t[chunks] = total tiles);
+// chunk_b[2 c] is the sequence that tile belongs to and chunk_b[2 c + 1] the
+// index of that piece among its sequence's pieces (0 when the chunk starts at
+// the sequence's first tile).
 struct WsLayout {
   size_t header = 0, tile_prefix = 0, split_base = 0, chunk_t = 0, chunk_b = 0, part_lse = 0,
          part_u = 0, total = 0;
@@ -56,6 +59,8 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_plan(const DecodeArgs& a, cudaStream_t s);
+// one bounded mbarrier wait, on a phase that completes (arrive) or never does
+cudaError_t launch_wait_selftest(int* err, bool arrive, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 
 // Tensor-core decode for small latent widths (one CTA per KV chunk and query

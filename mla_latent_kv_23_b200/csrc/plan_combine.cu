@@ -1,15 +1,25 @@
 // Plan and combine stages of mla_decode.
 //
 // plan:    per-sequence tile counts and their prefix sum; the cut of the tile
-//          line into KV chunks (uniform on a line that charges every sequence
-//          start kSegCostTiles units, so a chunk that starts new sequences
-//          takes fewer tiles); the first tile and sequence of every chunk; and
-//          the first partial row of every sequence that is cut into several
-//          chunks (one block; B is small).
+//          line into KV chunks; the first tile, sequence and piece index of
+//          every chunk; and the first partial row of every sequence that is
+//          cut into several chunks (one block; B is small).  Two cuts:
+//          * aligned: when every sequence has the same tile count t and the
+//            chunks divide among the sequences (c = chunks / B pieces each),
+//            sequence b takes chunks [c b, c b + c), piece k its tiles
+//            [k t / c, (k + 1) t / c): no chunk holds two sequences;
+//          * line: uniform on a line that charges every sequence start
+//            kSegCostTiles units, so a chunk that starts new sequences takes
+//            fewer tiles.
+//          The aligned cut is taken when its largest chunk is no bigger than
+//          the line's units per chunk plus one start charge (a chunk that
+//          holds two sequences pays a second query load and epilogue, which
+//          the charge only estimates).
 // combine: for every row cut into pieces, merge the partial results by their
 //          log-sum-exp: lse = log sum_s exp(lse_s), u = sum_s exp(lse_s - lse) u_s
 //          (the split-KV merge of softmax attention; exact up to rounding).
 #include <cuda_bf16.h>
+#include <limits.h>
 #include <math.h>
 
 #include "internal.h"
@@ -59,8 +69,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   ptx::pdl_launch_dependents();
   __shared__ int warp_sums[32];
   __shared__ int tp_s[kPlanSmemSeqs + 1];
+  __shared__ int tiles_min, tiles_max;
   const bool on_chip = B <= kPlanSmemSeqs;
   constexpr int K = kSegCostTiles;
+  if (threadIdx.x == 0) {
+    tiles_min = INT_MAX;
+    tiles_max = 0;
+  }
+  __syncthreads();
   int carry = 0, total = 0;
   for (int base = 0; base < B; base += blockDim.x) {
     const int i = base + threadIdx.x;
@@ -69,6 +85,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
       const int L = seqlens[i];
       if (L < s_q || L > max_len) atomicOr(err, MLA_DEVFLAG_BAD_SEQLEN);
       else tiles = (L + kTileTokens - 1) / kTileTokens;
+      atomicMin(&tiles_min, tiles);
+      atomicMax(&tiles_max, tiles);
     }
     const int incl = block_scan(tiles, warp_sums, &total);
     if (i < B) {
@@ -83,6 +101,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   // t + K (b + 1)
   const long long V = (long long)T + (long long)K * B;
   const int units = V > 0 ? (int)((V + num_chunks - 1) / num_chunks) : 1;
+  // the aligned cut: c pieces per sequence of t_seq tiles
+  const int t_seq = tiles_max;
+  const int cps = B > 0 ? min(num_chunks / B, t_seq) : 0;
+  const bool aligned = B > 0 && tiles_min == tiles_max && t_seq > 0 && cps >= 1 &&
+                       (t_seq + cps - 1) / cps <= units + K;
   if (threadIdx.x == 0) {
     tile_prefix[B] = T;
     if (on_chip) tp_s[B] = T;
@@ -90,22 +113,35 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
   __syncthreads();
   // the searches below read the prefix from shared memory when it fits
   const int* tp = on_chip ? tp_s : tile_prefix;
-  // chunk c starts at unit c * units: at the first tile at or after it
   for (int c = threadIdx.x; c <= num_chunks; c += blockDim.x) {
-    const long long x = (long long)c * units;
-    int t = T, sb = B;
-    if (x < V) {
-      int lo = 0, hi = B;  // largest b with tp[b] + K b <= x
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if ((long long)tp[mid] + (long long)K * mid <= x) lo = mid; else hi = mid;
+    int t = T, sb = B, part = 0;
+    if (aligned) {
+      if (c < B * cps) {
+        sb = c / cps;
+        part = c % cps;
+        t = tp[sb] + (int)((long long)part * t_seq / cps);
       }
-      const long long off = x - ((long long)tp[lo] + (long long)K * (lo + 1));
-      t = tp[lo] + (off > 0 ? (int)off : 0);
-      sb = lo;
+    } else {
+      // chunk c starts at unit c * units: at the first tile at or after it
+      const long long x = (long long)c * units;
+      if (x < V) {
+        int lo = 0, hi = B;  // largest b with tp[b] + K b <= x
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if ((long long)tp[mid] + (long long)K * mid <= x) lo = mid; else hi = mid;
+        }
+        const long long off = x - ((long long)tp[lo] + (long long)K * (lo + 1));
+        t = tp[lo] + (off > 0 ? (int)off : 0);
+        sb = lo;
+        // pieces of sequence lo are numbered from the chunk of its first tile
+        if (t > tp[lo]) part = c - (int)(((long long)tp[lo] + (long long)K * (lo + 1)) / units);
+      }
     }
     chunk_t[c] = t;
-    if (c < num_chunks) chunk_b[c] = sb;
+    if (c < num_chunks) {
+      chunk_b[2 * c] = sb;
+      chunk_b[2 * c + 1] = part;
+    }
   }
   carry = 0;
   for (int base = 0; base < B; base += blockDim.x) {
@@ -113,7 +149,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
     int pieces = 0;
     if (i < B) {
       const int t0 = tp[i], t1 = tp[i + 1];
-      if (t1 > t0) {
+      if (aligned) {
+        pieces = cps > 1 ? cps : 0;
+      } else if (t1 > t0) {
         const long long u0 = (long long)t0 + (long long)K * (i + 1);
         const int n = (int)((u0 + (t1 - t0) - 1) / units - u0 / units) + 1;
         pieces = n > 1 ? n : 0;
@@ -130,6 +168,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
     header[2] = num_chunks;
     header[3] = carry * s_q;
     header[4] = K;
+    header[5] = aligned ? 1 : 0;
   }
 }
 

@@ -2,13 +2,10 @@
 //
 // The plan stage lays every sequence's 64-token tiles end to end
 // (tile_prefix[b] = first tile of sequence b) and cuts that line into chunks;
-// chunk c holds tiles [chunk_t[c], chunk_t[c + 1]).  The cuts are uniform on
-// a line where every sequence takes K units of start-up cost before its tiles
-// (units [tile_prefix[b] + K b, tile_prefix[b] + K (b + 1))), so tile t of
-// sequence b sits at unit t + K (b + 1) and lies in chunk
-// (t + K (b + 1)) / units_per_chunk.  A chunk
-// can cover the tail of one sequence, some whole sequences and the head of
-// another; each piece is a segment.  A segment that covers a whole sequence
+// chunk c holds tiles [chunk_t[c], chunk_t[c + 1]) (the plan kernel says how
+// the cuts are placed).  A chunk can cover the tail of one sequence, some
+// whole sequences and the head of another; each piece is a segment, and the
+// pieces of a sequence are numbered in tile order.  A segment that covers a whole sequence
 // writes u/lse directly; otherwise it writes a partial row that the combine
 // stage merges.  Every role of every CTA walks the same segments in the same
 // order.
@@ -26,22 +23,21 @@ struct Segment {
 struct ChunkWalk {
   const int* tp;  // tile_prefix, B + 1 entries
   int B;
-  int t, t_end, chunk, b;
-  int units, K;  // line units per chunk, units per sequence start
+  int t, t_end, b;
+  int part0;  // piece index of the chunk's first segment
 
-  // chunk_t / chunk_b / header come from the plan stage; the three reads are
-  // independent (one memory round trip)
+  // chunk_t / chunk_b come from the plan stage; the reads are independent
+  // (one memory round trip)
   __device__ __forceinline__ void init(const int* tile_prefix, const int* chunk_t,
                                        const int* chunk_b, const int* header, int nseq,
                                        int chunk_id) {
+    (void)header;
     tp = tile_prefix;
     B = nseq;
-    chunk = chunk_id;
     t = chunk_t[chunk_id];
     t_end = chunk_t[chunk_id + 1];
-    b = chunk_b[chunk_id];
-    units = header[1];
-    K = header[4];
+    b = chunk_b[2 * chunk_id];
+    part0 = chunk_b[2 * chunk_id + 1];
   }
 
   __device__ __forceinline__ bool next(Segment& s) {
@@ -54,8 +50,8 @@ struct ChunkWalk {
     s.t0 = t - begin;
     s.t1 = stop - begin;
     s.whole = (t == begin && stop == end) ? 1 : 0;
-    // pieces of sequence b are numbered from the chunk holding its first tile
-    s.part = chunk - (int)(((long long)begin + (long long)K * (b + 1)) / units);
+    // a later segment of the chunk starts its sequence: piece 0
+    s.part = t == begin ? 0 : part0;
     t = stop;
     return true;
   }

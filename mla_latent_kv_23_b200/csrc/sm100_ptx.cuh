@@ -103,14 +103,15 @@ __device__ __forceinline__ bool mbar_test_nb_cluster(uint32_t bar, uint32_t pari
 // was measured to add hundreds of ns of wake-up latency to hand-offs between
 // warps of this kernel, even for phases that had already completed.
 template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int flag,
+                                          uint64_t limit = kWaitLimitCycles) {
   if (kCluster ? mbar_test_nb_cluster(bar, parity) : mbar_test_nb(bar, parity)) return true;
   const uint64_t t0 = cycles();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (kCluster ? mbar_test_nb_cluster(bar, parity) : mbar_test_nb(bar, parity)) return true;
-    if (cycles() - t0 > kWaitLimitCycles) {
+    if (cycles() - t0 > limit) {
       atomicOr(err, flag);
       return false;
     }

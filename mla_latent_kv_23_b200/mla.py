@@ -78,6 +78,7 @@ SIGNATURES = {
     "mla_up_proj": ([_V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
     "mla_merge_partials": ([_V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
     "mla_check_device_errors": ([_V, ctypes.POINTER(_I)], _I),
+    "mla_selftest_wait": ([_I, _V], _I),
 }
 
 _lib = None
@@ -350,6 +351,11 @@ def mla_check_device_errors(stream=None) -> int:
     if st != 0:
         raise MLAError("mla_check_device_errors", st, f.value)
     return f.value
+
+
+def mla_selftest_wait(arrive: bool, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see include/mla.h)."""
+    _check(lib().mla_selftest_wait(1 if arrive else 0, _stream(stream)), "mla_selftest_wait")
 
 
 def mla_status_string(status: int) -> str:

@@ -294,6 +294,29 @@ def test_device_flags_for_bad_inputs():
     assert mla.mla_check_device_errors() == 0   # flags were cleared
 
 
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    # the wait every kernel uses on its mbarriers: on a phase that completes
+    # it returns at once; on one that never completes it gives up after its
+    # limit, raises the timeout flag and the kernel ends; the next decode
+    # runs and agrees with one taken before
+    w = v3_small(B=2, seqlens=(100, 200), block_table="identity")
+    inp = synth.draw(w)
+    q = to_dev(synth.random_q(w), w)
+    cache, bt, sl = to_dev(inp["cache"], w), to_dev_i32(inp["block_table"]), to_dev_i32(inp["seqlens"])
+    u0, l0 = mla.decode(q, cache, bt, sl, w.page_size, w.d_R, w.softmax_scale)
+    assert mla.mla_check_device_errors() == 0
+    mla.mla_selftest_wait(True)
+    assert mla.mla_check_device_errors() == 0
+    mla.mla_selftest_wait(False)
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_check_device_errors()
+    assert e.value.flags == mla.DEVFLAG_TIMEOUT
+    assert mla.mla_check_device_errors() == 0   # flags were cleared
+    u1, l1 = mla.decode(q, cache, bt, sl, w.page_size, w.d_R, w.softmax_scale)
+    assert mla.mla_check_device_errors() == 0
+    assert torch.equal(u0, u1) and torch.equal(l0, l1)
+
+
 def test_empty_batch():
     q = torch.empty((0, 1, 128, 576), dtype=torch.bfloat16, device="cuda")
     cache = torch.zeros((64, 576), dtype=torch.bfloat16, device="cuda")
