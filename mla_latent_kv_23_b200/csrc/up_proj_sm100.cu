@@ -35,7 +35,10 @@ using namespace ptx;
 
 enum class UpMode { kBf16, kSplitU, kTf32 };
 
-constexpr int kThreads = 128;
+// 16 warps: the row loads and the partial merge are latency-bound (a few
+// dependent memory round trips per row), so each warp takes one row of a
+// 16-row block at a time; warps 0-3 drain the accumulator.
+constexpr int kThreads = 512;
 constexpr int kM = 128;              // MMA rows: d_v <= 128
 constexpr int kMaxKb = 8;            // 128-byte column blocks of d_c
 constexpr int kMaxRows = 64;         // query rows per CTA (kBf16, kTf32)
@@ -108,144 +111,189 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
     for (int kb = 0; kb < kb_n; ++kb)
       tma_load_2d(sbase + kb * kWBlk, &p.w_map, bar_w, kb * kColsPerBlk, head * p.d_v);
   }
-  pdl_wait_previous();
-  pdl_launch_dependents();
+  // kSplitU: the B operand holds 2 n_pad rows per 128-byte column block,
+  // row tt = bf16(u_t) (hi) and row n_pad + tt = bf16(u_t - hi) (lo), so
+  // one MMA chain over W gives W hi and W lo side by side (N = 2 n_pad)
+  const uint32_t ublk2 = 2 * ublk;
+  auto store_hilo = [&](int tt, int c8, const float (&v)[8]) {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+      const float2 hf = __bfloat1622float2(h2);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * k] - hf.x, v[2 * k + 1] - hf.y);
+      hi[k] = *reinterpret_cast<const uint32_t*>(&h2);
+      lo[k] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+    // chunk k16 of row r at byte r * 128 + ((k16 ^ (r & 7)) << 4) of its
+    // block; n_pad is a multiple of 16, so rows tt and n_pad + tt share it
+    const int kb = c8 >> 3, k16 = c8 & 7;
+    const uint32_t sw = static_cast<uint32_t>(k16 ^ (tt & 7)) << 4;
+    const uint32_t blk = sbase + off_u + kb * ublk2;
+    st_shared_v4(blk + tt * 128 + sw, hi[0], hi[1], hi[2], hi[3]);
+    st_shared_v4(blk + (p.n_pad + tt) * 128 + sw, lo[0], lo[1], lo[2], lo[3]);
+  };
   if constexpr (kMode == UpMode::kSplitU) {
    if (p.merge) {
-    // one warp per row t; lane l owns columns [16 l, 16 l + 16) of d_c = 512
-    for (int tt = warp; tt < p.n_pad; tt += kThreads / 32) {
-      const int t = t0 + tt;
+    // One warp per row t (rows warp and warp + 16 of the block); lane l
+    // owns columns [16 l, 16 l + 16) of d_c = 512.  The plan stage's
+    // outputs are read before the wait: the plan kernel completed before
+    // the attend kernel passed its own wait, and this kernel was launched
+    // only after every attend CTA had passed it.
+    constexpr int kRowsPerWarp = kMaxRowsSplit / (kThreads / 32);
+    int kind[kRowsPerWarp], sb0[kRowsPerWarp], nsp[kRowsPerWarp];  // kind: 0 none, 1 whole, 2 empty, 3 split
+#pragma unroll
+    for (int j = 0; j < kRowsPerWarp; ++j) {
+      const int tt = warp + j * (kThreads / 32), t = t0 + tt;
+      kind[j] = 0;
+      sb0[j] = 0;
+      nsp[j] = 0;
+      if (tt < p.n_pad && t < p.T) {
+        const int b = t / p.s_q;
+        const int s0 = p.split_base[b], s1 = p.split_base[b + 1];
+        const bool has_tokens = p.tile_prefix[b + 1] != p.tile_prefix[b];
+        sb0[j] = s0;
+        nsp[j] = s1 - s0;
+        kind[j] = s1 > s0 ? 3 : (has_tokens ? 1 : 2);
+      }
+    }
+    pdl_wait_previous();
+    pdl_launch_dependents();
+#pragma unroll
+    for (int j = 0; j < kRowsPerWarp; ++j) {
+      const int tt = warp + j * (kThreads / 32), t = t0 + tt;
+      if (tt >= p.n_pad) continue;
       float acc[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-      if (t < p.T) {
-        const int b = t / p.s_q, r = t % p.s_q;
-        const int sb0 = p.split_base[b], nsplit = p.split_base[b + 1] - sb0;
-        const size_t urow = (size_t)t * p.n_h + head;
-        float* up = p.u_out + urow * 512 + 16 * lane;
-        if (nsplit == 0) {
-          if (p.tile_prefix[b + 1] != p.tile_prefix[b]) {  // written whole by the attend stage
+      const size_t urow = (size_t)t * p.n_h + head;
+      float* up = p.u_out + urow * 512 + 16 * lane;
+      if (kind[j] == 1) {  // written whole by the attend stage
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float4 v = reinterpret_cast<const float4*>(up)[i];
-              acc[4 * i] = v.x; acc[4 * i + 1] = v.y; acc[4 * i + 2] = v.z; acc[4 * i + 3] = v.w;
-            }
-          } else {  // no tokens (a rejected length): u = 0, lse = -inf
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = reinterpret_cast<const float4*>(up)[i];
+          acc[4 * i] = v.x; acc[4 * i + 1] = v.y; acc[4 * i + 2] = v.z; acc[4 * i + 3] = v.w;
+        }
+      } else if (kind[j] == 2) {  // no tokens (a rejected length): u = 0, lse = -inf
 #pragma unroll
-            for (int i = 0; i < 4; ++i) reinterpret_cast<float4*>(up)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (lane == 0 && p.lse_out) p.lse_out[urow] = -INFINITY;
+        for (int i = 0; i < 4; ++i) reinterpret_cast<float4*>(up)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0 && p.lse_out) p.lse_out[urow] = -INFINITY;
+      } else if (kind[j] == 3) {
+        const int nsplit = nsp[j];
+        const size_t slot0 = (size_t)sb0[j] * p.s_q + t % p.s_q;  // slot of split s: slot0 + s s_q
+        auto lse_of = [&](int sp) { return p.part_lse[(slot0 + (size_t)sp * p.s_q) * p.n_h + head]; };
+        auto part_of = [&](int sp) {
+          return reinterpret_cast<const float4*>(
+              p.part_u + ((slot0 + (size_t)sp * p.s_q) * p.n_h + head) * 512 + 16 * lane);
+        };
+        // the first four partial rows are requested together with the
+        // statistics: one memory round trip for rows of up to four pieces
+        float4 v[4][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k < nsplit) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[k][i] = part_of(k)[i];
           }
-        } else {
-          const size_t slot0 = (size_t)sb0 * p.s_q + r;  // slot of split s: slot0 + s s_q
-          auto lse_of = [&](int sp) { return p.part_lse[(slot0 + (size_t)sp * p.s_q) * p.n_h + head]; };
-          float m = -INFINITY, z = 0.f;
-          for (int sp = lane; sp < nsplit; sp += 32) {
-            const float x = lse_of(sp);
-            if (x > m) {
-              z = z * expf(m - x) + 1.f;
-              m = x;
-            } else if (x != -INFINITY) {
-              z += expf(x - m);
-            }
+        const float x_lane = lane < nsplit ? lse_of(lane) : -INFINITY;
+        float m = x_lane, z = x_lane == -INFINITY ? 0.f : 1.f;
+        for (int sp = lane + 32; sp < nsplit; sp += 32) {
+          const float x = lse_of(sp);
+          if (x > m) {
+            z = z * expf(m - x) + 1.f;
+            m = x;
+          } else if (x != -INFINITY) {
+            z += expf(x - m);
           }
-          float m_all = m;
+        }
+        float m_all = m;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m_all = fmaxf(m_all, __shfl_xor_sync(0xffffffffu, m_all, o));
-          z = m == -INFINITY ? 0.f : z * expf(m - m_all);
+        for (int o = 16; o > 0; o >>= 1) m_all = fmaxf(m_all, __shfl_xor_sync(0xffffffffu, m_all, o));
+        z = m == -INFINITY ? 0.f : z * expf(m - m_all);
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-          const float lse = m_all == -INFINITY ? -INFINITY : m_all + logf(z);
-          if (m_all != -INFINITY) {
-            for (int s0 = 0; s0 < nsplit; s0 += 4) {
-              float4 v[4][4];
-              const int n_here = min(4, nsplit - s0);
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        const float lse = m_all == -INFINITY ? -INFINITY : m_all + logf(z);
+        if (m_all != -INFINITY) {
+          const float w_lane = x_lane == -INFINITY ? 0.f : expf(x_lane - lse);
+          for (int s0 = 0; s0 < nsplit; s0 += 4) {
+            const int n_here = min(4, nsplit - s0);
+            if (s0 > 0) {
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 if (k < n_here) {
-                  const float4* src = reinterpret_cast<const float4*>(
-                      p.part_u + ((slot0 + (size_t)(s0 + k) * p.s_q) * p.n_h + head) * 512 + 16 * lane);
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) v[k][i] = src[i];
+                  for (int i = 0; i < 4; ++i) v[k][i] = part_of(s0 + k)[i];
                 }
-              const float w_me = lane < n_here ? expf(lse_of(s0 + lane) - lse) : 0.f;
+            }
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float w = __shfl_sync(0xffffffffu, w_me, k);
-                if (k < n_here) {
+            for (int k = 0; k < 4; ++k) {
+              // split s0 + k's weight: held by lane s0 + k for the first 32
+              const float wk = s0 + k < 32 ? __shfl_sync(0xffffffffu, w_lane, (s0 + k) & 31) : 0.f;
+              const float w = s0 + k < 32 ? wk : (k < n_here ? expf(lse_of(s0 + k) - lse) : 0.f);
+              if (k < n_here) {
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    acc[4 * i] += w * v[k][i].x;
-                    acc[4 * i + 1] += w * v[k][i].y;
-                    acc[4 * i + 2] += w * v[k][i].z;
-                    acc[4 * i + 3] += w * v[k][i].w;
-                  }
+                for (int i = 0; i < 4; ++i) {
+                  acc[4 * i] += w * v[k][i].x;
+                  acc[4 * i + 1] += w * v[k][i].y;
+                  acc[4 * i + 2] += w * v[k][i].z;
+                  acc[4 * i + 3] += w * v[k][i].w;
                 }
               }
             }
           }
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            reinterpret_cast<float4*>(up)[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-          if (lane == 0 && p.lse_out) p.lse_out[urow] = lse;
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(up)[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        if (lane == 0 && p.lse_out) p.lse_out[urow] = lse;
       }
       // the row's two bf16 terms: lane l's 16 columns are chunks 2l, 2l + 1
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t hi[4], lo[4];
+        float v8[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float a0 = acc[8 * c + 2 * k], a1 = acc[8 * c + 2 * k + 1];
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
-          const float2 hf = __bfloat1622float2(h2);
-          const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
-          hi[k] = *reinterpret_cast<const uint32_t*>(&h2);
-          lo[k] = *reinterpret_cast<const uint32_t*>(&l2);
-        }
-        const int c8 = 2 * lane + c, kb = c8 >> 3, k16 = c8 & 7;
-        const uint32_t off = kb * ublk + tt * 128 + ((static_cast<uint32_t>(k16 ^ (tt & 7))) << 4);
-        st_shared_v4(sbase + off_u + off, hi[0], hi[1], hi[2], hi[3]);
-        st_shared_v4(sbase + off_u + kMaxKb * ublk + off, lo[0], lo[1], lo[2], lo[3]);
+        for (int k = 0; k < 8; ++k) v8[k] = acc[8 * c + k];
+        store_hilo(tt, 2 * lane + c, v8);
       }
     }
     fence_proxy_async_smem();
     __syncthreads();
    } else {
+    pdl_wait_previous();
+    pdl_launch_dependents();
     // u rows -> hi and lo bf16 terms, 8 columns (one 16-byte chunk of each
-    // term) per step, in the 128-byte swizzle the MMA descriptor expects:
-    // chunk k of row t at byte t * 128 + ((k ^ (t & 7)) << 4) of its block;
-    // rows past T are zero
-    const int chunks = p.d_c / 8;
-    for (int unit = threadIdx.x; unit < p.n_pad * chunks; unit += kThreads) {
-      const int t = unit / chunks, c8 = unit % chunks;
-      float v[8];
-      if (t0 + t < p.T) {
-        const float4* src = reinterpret_cast<const float4*>(
-            p.u_f32 + ((size_t)(t0 + t) * p.n_h + head) * p.d_c + 8 * c8);
-        const float4 a = src[0], b = src[1];
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = 0.f;
-      }
-      uint32_t hi[4], lo[4];
+    // term) per unit; each thread requests up to four units' rows before
+    // using any; rows past T are zero
+    const int chunks = p.d_c / 8, units = p.n_pad * chunks;
+    for (int base_u = 0; base_u < units; base_u += 4 * kThreads) {
+      float v[4][8];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-        const float2 hf = __bfloat1622float2(h2);
-        const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * k] - hf.x, v[2 * k + 1] - hf.y);
-        hi[k] = *reinterpret_cast<const uint32_t*>(&h2);
-        lo[k] = *reinterpret_cast<const uint32_t*>(&l2);
+        const int unit = base_u + k * kThreads + threadIdx.x;
+        const int t = unit / chunks, c8 = unit % chunks;
+        if (unit < units && t0 + t < p.T) {
+          const float4* src = reinterpret_cast<const float4*>(
+              p.u_f32 + ((size_t)(t0 + t) * p.n_h + head) * p.d_c + 8 * c8);
+          const float4 a = src[0], b = src[1];
+          v[k][0] = a.x; v[k][1] = a.y; v[k][2] = a.z; v[k][3] = a.w;
+          v[k][4] = b.x; v[k][5] = b.y; v[k][6] = b.z; v[k][7] = b.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[k][i] = 0.f;
+        }
       }
-      const int kb = c8 >> 3, k16 = c8 & 7;
-      const uint32_t off = kb * ublk + t * 128 + ((static_cast<uint32_t>(k16 ^ (t & 7))) << 4);
-      st_shared_v4(sbase + off_u + off, hi[0], hi[1], hi[2], hi[3]);
-      st_shared_v4(sbase + off_u + kMaxKb * ublk + off, lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int unit = base_u + k * kThreads + threadIdx.x;
+        if (unit < units) store_hilo(unit / chunks, unit % chunks, v[k]);
+      }
     }
     fence_proxy_async_smem();
     __syncthreads();
    }
+  } else {
+    pdl_wait_previous();
+    pdl_launch_dependents();
   }
   bool ok = true;
   if (threadIdx.x == 0) {
@@ -258,14 +306,15 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
     ok = ok && mbar_wait(bar_w, 0, p.err, MLA_DEVFLAG_TIMEOUT);
     if (ok) {
       tc_fence_after();
-      const uint32_t idesc = kF32 ? idesc_tf32(kM, p.n_pad, false) : idesc_bf16(kM, p.n_pad, false);
+      constexpr bool kTwo = kMode == UpMode::kSplitU;  // hi and lo side by side in N
+      const int n_mma = kTwo ? 2 * p.n_pad : p.n_pad;
+      const uint32_t bblk = kTwo ? ublk2 : ublk;
+      const uint32_t idesc = kF32 ? idesc_tf32(kM, n_mma, false) : idesc_bf16(kM, n_mma, false);
       uint32_t acc = 0;
-      for (int term = 0; term < (kMode == UpMode::kSplitU ? 2 : 1); ++term)
         for (int kb = 0; kb < kb_n; ++kb)
           for (int ks = 0; ks < 4; ++ks) {  // 32 bytes of K per instruction
             const uint64_t a = smem_desc(sbase + kb * kWBlk + ks * 32, 16, 1024, kLayoutSW128);
-            const uint64_t b = smem_desc(sbase + off_u + (term * kMaxKb + kb) * ublk + ks * 32, 16,
-                                         1024, kLayoutSW128);
+            const uint64_t b = smem_desc(sbase + off_u + kb * bblk + ks * 32, 16, 1024, kLayoutSW128);
             if (kF32)
               umma_tf32_ss(tmem, a, b, idesc, acc);
             else
@@ -278,13 +327,20 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
   }
   ok = __syncthreads_and(ok);
   tc_fence_after();
-  if (ok) {
+  if (ok && warp < 4) {
     // thread (warp w, lane l) owns output row v = 32 w + l; columns are rows t
     const int v = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     for (int c0 = 0; c0 < p.n_pad; c0 += 32) {
       float d[32];
       tmem_ld32(tmem + lane_base + c0, d);
+      if constexpr (kMode == UpMode::kSplitU) {  // W hi + W lo
+        float e[32];
+        tmem_ld32(tmem + lane_base + p.n_pad + c0, e);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) d[k] += e[k];
+      }
       tmem_wait_ld();
       if (v < p.d_v) {
 #pragma unroll
