@@ -296,11 +296,13 @@ def run_gpu(args, w):
                 return
             mla.mla_decode(p, ws)
         else:
+            ev[2].record()
             mla.mla_decode_plan(p, ws)
             ev[0].record()
             mla.mla_decode_attend(p, ws)
             ev[1].record()
             mla.mla_decode_combine(p, ws)
+            ev[3].record()
         mla.mla_up_proj(u.view(T, w.n_h, w.d_c), W_UV, o)
 
     # direct launches once (initialises the library, checks flags)
@@ -320,8 +322,8 @@ def run_gpu(args, w):
             step(i)
         graphs.append(g)
         g = torch.cuda.CUDAGraph()
-        ev = (torch.cuda.Event(enable_timing=True, external=True),
-              torch.cuda.Event(enable_timing=True, external=True))
+        # [0, 1] around the attend kernel, [2, 3] around plan + attend + combine
+        ev = tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(4))
         with torch.cuda.graph(g, stream=stream):
             step(i, ev)
         timed_graphs.append(g)
@@ -388,6 +390,8 @@ def run_gpu(args, w):
     mla.mla_check_device_errors(stream)
     ms_total = t_start.elapsed_time(t_end)
     attend_ms = statistics.fmean(evs[i][0].elapsed_time(evs[i][1]) for i in ev_copies)
+    decode_ms = statistics.fmean(evs[i][2].elapsed_time(evs[i][3]) for i in ev_copies)
+    hdr = ws[:64 * 4].view(torch.int32).cpu().tolist()  # the plan's header (workspace)
 
     t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
     if world > 1:
@@ -419,6 +423,10 @@ def run_gpu(args, w):
     roof["roofline_us"] = max(t_hbm, t_tc) * 1e6
     roof["alg_bytes_per_launch"] = dw["bytes"]
     roof["alg_flops_per_launch"] = dw["flops"]
+    # the decode stage alone (plan + attend + combine, staged calls with
+    # events around them), against the same roofline
+    decode_stage = {"us": decode_ms * 1e3, "frac": max(t_hbm, t_tc) / (decode_ms * 1e-3),
+                    "calls": "mla_decode_plan + mla_decode_attend + mla_decode_combine"}
 
     # ---- end to end through the public API with host buffers (pinned)
     e2e = run_e2e(args, w, inp, q0, bt, sl, W_UV, dev, stream, mla, step_flops, world) \
@@ -442,12 +450,15 @@ def run_gpu(args, w):
                 "us_per_step": ms_step * 1e3,
                 "hbm_gbs": world * step_bytes / (ms_step * 1e-3) / 1e9,
                 "decode_roofline_frac_step": max(t_hbm, t_tc) * 1e3 / ms_step,
-                "kv_chunks": chunks,
+                "kv_chunks": chunks, "kv_chunks_used": int(hdr[6]),
+                "kv_cut": "aligned to sequences" if int(hdr[5]) else "cost line",
+                "decode_stage": decode_stage,
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": (3 if fused else 4) * (args.steps - n_ev) + 4 * n_ev, "clocks": clocks}
         print(json.dumps(line), flush=True)
     graphs.clear()
     timed_graphs.clear()
+    del chain
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -22,7 +22,8 @@ constexpr int kSegCostTiles = 4;
 
 // Workspace of mla_decode.  Header ints: [0] total tiles, [1] line units per
 // chunk, [2] number of chunks, [3] split rows in use, [4] units per sequence
-// start, [5] 1 when the chunks follow the sequences (see the plan kernel).
+// start, [5] 1 when the chunks follow the sequences (see the plan kernel),
+// [6] the chunks in use (the others are empty).
 // chunk_t[c] is the first tile of chunk c (chunk_t[chunks] = total tiles);
 // chunk_b[2 c] is the sequence that tile belongs to and chunk_b[2 c + 1] the
 // index of that piece among its sequence's pieces (0 when the chunk starts at

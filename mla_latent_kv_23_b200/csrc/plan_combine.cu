@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
     header[3] = carry * s_q;
     header[4] = K;
     header[5] = aligned ? 1 : 0;
+    header[6] = aligned ? B * cps : num_chunks;  // chunks that hold tiles (at most)
   }
 }
 
