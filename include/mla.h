@@ -60,6 +60,7 @@ typedef enum { MLA_DTYPE_BF16 = 0, MLA_DTYPE_FP32 = 1 } mla_dtype;
 #define MLA_DEVFLAG_BAD_PAGE 0x2    /* block_table entry outside [0, num_pages) */
 #define MLA_DEVFLAG_TIMEOUT 0x4     /* a device-side wait gave up (kernel returned early) */
 #define MLA_DEVFLAG_LAYOUT 0x8      /* a kernel's shared memory was not 1024-byte aligned (it returned at once) */
+#define MLA_DEVFLAG_RANGE 0x10      /* a split row's partial u did not fit fp16 (|value| > 65504): u of that row is wrong */
 
 const char* mla_status_string(mla_status s);
 
@@ -190,7 +191,9 @@ typedef struct {
   float softmax_scale;      /* multiplies the scores before softmax, finite and > 0               */
   mla_dtype dtype;          /* of q, kv_cache and u                                              */
   int num_splits;           /* KV chunks the whole batch is cut into; 0 = one per SM pair        */
-  int u_fp32;               /* nonzero: u (and the partial results of split rows) are fp32;
+  int u_fp32;               /* nonzero: u is fp32 (the partial u of pieces of split rows fp16 on the
+                               DeepSeek-V3-shape kernel, which flags MLA_DEVFLAG_RANGE if a value
+                               exceeds 65504; fp32 on the small-latent kernel);
                                0: u has type `dtype`.  With bf16 inputs an fp32 u carries the
                                softmax-weighted latent sum to the up-projection unrounded: a
                                bf16 u moves o = W_UV u by up to 2^-8 |u| per element, which for
@@ -230,7 +233,7 @@ mla_status mla_decode_combine(const mla_decode_params* p, void* workspace,
 /*
  * One decode step of the attention output: mla_decode, then o = W_UV u
  * (as mla_up_proj), with the combine of split rows done inside the
- * up-projection: each up-projection CTA merges the fp32 partials of its
+ * up-projection: each up-projection CTA merges the fp16 partials of its
  * head's rows from the workspace (also writing u and lse), splits the fp32
  * rows into two bf16 terms and runs the tensor-core product.  The three
  * kernels (plan, attend, merge + up-projection) are chained by programmatic

@@ -186,6 +186,7 @@ mla_status resolve(const mla_decode_params* p, void* ws, size_t ws_bytes, Resolv
   a.bf16 = p->dtype == MLA_DTYPE_BF16;
   a.out_f32 = p->u_fp32 != 0 || p->dtype == MLA_DTYPE_FP32;
   a.part_bf16 = r->kernel == Kernel::kV3 && !a.out_f32;
+  a.part_f16 = r->kernel == Kernel::kV3 && a.out_f32;
   a.pdl = false;
   return MLA_OK;
 }
@@ -291,18 +292,22 @@ mla_status encode_q(CUtensorMap* m, const void* ptr, uint64_t n_h, uint64_t qrow
 }
 
 // 3D map over an output [rows, n_h, 512] for TMA stores, 128-byte swizzle:
-// bf16 with boxes of 64 columns x 32 heads x 1, or fp32 with boxes of 32
-// columns x 32 heads x 1 (one 128-byte line per head either way).
-mla_status encode_out(CUtensorMap* m, void* ptr, uint64_t n_h, uint64_t rows, bool f32) {
+// 16-bit (bf16 or fp16) with boxes of 64 columns x 32 heads x 1, or fp32 with
+// boxes of 32 columns x 32 heads x 1 (one 128-byte line per head either way).
+enum class OutType { kBf16, kF16, kF32 };
+mla_status encode_out(CUtensorMap* m, void* ptr, uint64_t n_h, uint64_t rows, OutType t) {
+  const bool f32 = t == OutType::kF32;
   const uint64_t es = f32 ? 4 : 2;
   const cuuint64_t dims[3] = {512, n_h, rows};
   const cuuint64_t strides[2] = {512 * es, n_h * 512 * es};
   const cuuint32_t box[3] = {f32 ? 32u : 64u, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                        3, ptr, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                     : (t == OutType::kF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  CUresult r = g_encode(m, dt, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -359,8 +364,10 @@ mla_status attend(Resolved r, const mla_decode_params* p, cudaStream_t s, bool p
   maps.has_kv4 = encode_kv_lat4(&maps.kv_lat4, p->kv_cache, kvrows) ? 1 : 0;
   maps.has_q5 = p->n_h % 16 == 0 && encode_q5(&maps.q_lat5, p->q, p->n_h, qrows, false) &&
                 encode_q5(&maps.q_rope5, p->q, p->n_h, qrows, true);
-  if ((st = encode_out(&maps.u_out, p->u, p->n_h, qrows, r.a.out_f32)) != MLA_OK ||
-      (st = encode_out(&maps.part_out, r.a.part_u, p->n_h, (uint64_t)r.slots, r.a.out_f32)) !=
+  if ((st = encode_out(&maps.u_out, p->u, p->n_h, qrows,
+                       r.a.out_f32 ? OutType::kF32 : OutType::kBf16)) != MLA_OK ||
+      (st = encode_out(&maps.part_out, r.a.part_u, p->n_h, (uint64_t)r.slots,
+                       r.a.part_f16 ? OutType::kF16 : OutType::kBf16)) !=
           MLA_OK)
     return st;
   return cuda_status(launch_decode_sm100(r.a, maps, s));
@@ -825,6 +832,7 @@ mla_status mla_decode_gqa(const mla_gqa_params* p, void* ws, size_t ws_bytes, vo
   a.bf16 = true;
   a.out_f32 = p->o_fp32 != 0;
   a.part_bf16 = false;
+  a.part_f16 = false;
   a.pdl = false;
   const int hpg = p->n_h / p->n_g;
   const uint64_t wq = (uint64_t)p->d_h + p->d_R, wkv = (uint64_t)p->d_h + p->d_v;

@@ -58,12 +58,16 @@
 //
 // Epilogue: u = O / l leaves TMEM through the query area (free once the
 // segment's last S is done) by TMA stores of whole 128-byte lines; the relay
-// loads the next segment's query after those stores have read it.
+// loads the next segment's query after those stores have read it.  u is fp32
+// or bf16; the partial u of a piece of a split sequence is fp16 with an fp32
+// u (bf16 with a bf16 u).
 //
-// Work: the plan stage cuts the batch's tiles into chunks of equal cost
-// (tiles plus a fixed charge per sequence start); cluster c handles chunk
+// Work: the plan stage cuts the batch's tiles into chunks (following the
+// sequences when their lengths are equal, else of equal cost on a line that
+// charges every sequence start); cluster c handles chunk
 // c / s_q for query row c % s_q, walking its segments in order.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "internal.h"
@@ -152,7 +156,7 @@ struct Params {
   float* lse;
   int* err;
   int B, s_q, n_h, max_pages, page_size, num_pages;
-  int out_f32;       // u and the split partials are fp32 (else bf16)
+  int out_f32;       // u is fp32, its split partials fp16 (else both bf16)
   float scale_log2;  // softmax_scale * log2(e)
 };
 
@@ -756,7 +760,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int col0 = 256 * c + 128 * (qd >> 1);  // latent column of TMEM column kTmemO + 128c
       // The segment's last S has read Q, so the query area stages the output:
       // 8 KB per warp, its 32 heads x 128 columns as boxes of 128-byte lines
-      // (64 bf16 or 32 fp32 columns) in the 128-byte-swizzled layout of the
+      // (64 16-bit or 32 fp32 columns) in the 128-byte-swizzled layout of the
       // output tensor map (row = head = lane, 16-byte chunk k of a row at
       // k ^ (row & 7)).  Each box leaves by one TMA store, which writes whole
       // 128-byte lines of u; the relay loads the next segment's query only
@@ -764,7 +768,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t stg = sbase + kOffQ + sw_warp * 8192u;
       const int y_head = 64 * (int)rank + 32 * (qd & 1);  // first head of this warp's rows
       const CUtensorMap* omap = sg.whole ? &p.maps.u_out : &p.maps.part_out;
-      if (p.out_f32) {
+      if (p.out_f32 && sg.whole) {
         // fp32: four boxes of 32 columns (one 128-byte line per head), two
         // at a time through the warp's 8 KB
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -789,21 +793,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
       } else {
+        bool f16_range_ok = true;  // fp16 partials: every value fits
         for (int c0 = 0; c0 < 128; c0 += 32) {
           float o[32];
           tmem_ld32(tmem + lane_base + kTmemO + c * 128 + c0, o);
           tmem_wait_ld();
-          // u of a whole sequence, or this segment's partial u (the combine
-          // stage weights and sums the partials in fp32): bf16 either way
+          // 16-bit rows: with a bf16 u, u of a whole sequence or this
+          // segment's partial u, both bf16; with an fp32 u, the partial u in
+          // fp16 (the merge weights and sums the partials in fp32)
           const uint32_t row = stg + static_cast<uint32_t>(c0 >> 6) * 4096u + lane * 128u;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             uint32_t w[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const __nv_bfloat162 h2 =
-                  __floats2bfloat162_rn(o[8 * e + 2 * k] * inv, o[8 * e + 2 * k + 1] * inv);
-              w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+              const float x0 = o[8 * e + 2 * k] * inv, x1 = o[8 * e + 2 * k + 1] * inv;
+              if (p.out_f32) {
+                const __half2 h2 = __floats2half2_rn(x0, x1);
+                w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+                f16_range_ok &= fabsf(x0) <= 65504.f && fabsf(x1) <= 65504.f;
+              } else {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+                w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
             }
             const uint32_t chunk16 = static_cast<uint32_t>(((c0 & 63) >> 3) + e);
             st_shared_v4(row + ((chunk16 ^ static_cast<uint32_t>(lane & 7)) << 4), w[0], w[1],
@@ -819,6 +831,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         }
+        if (!__all_sync(0xffffffffu, f16_range_ok) && lane == 0) atomicOr(p.err, MLA_DEVFLAG_RANGE);
       }
       const int head = 64 * (int)rank + hO;
       if (head < p.n_h && qd < 2 && c == 0) {

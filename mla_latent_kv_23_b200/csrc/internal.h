@@ -55,7 +55,8 @@ struct DecodeArgs {
   float scale;
   bool bf16;       // q and the cache are bf16 (else fp32)
   bool out_f32;    // u is fp32 (else bf16)
-  bool part_bf16;  // split partials of u are bf16 (exactly when u is bf16)
+  bool part_bf16;  // split partials of u are bf16 (the DeepSeek-V3-shape kernel with a bf16 u)
+  bool part_f16;   // split partials of u are fp16 (that kernel with an fp32 u); else fp32
   bool pdl;        // launch as a programmatic dependent of the previous kernel
 };
 
@@ -157,7 +158,7 @@ cudaError_t launch_up_proj_sm100(const CUtensorMap& w_map, const CUtensorMap& u_
 // bf16 W and o with an fp32 u, read with plain loads and split into two bf16
 // terms, u = hi + lo, in shared memory: o = W^UV hi + W^UV lo.  With
 // `merge` (d_c = 512), the rows of split sequences are first merged from the
-// decode workspace's fp32 partials (and written to u and lse): the combine
+// decode workspace's fp16 partials (and written to u and lse): the combine
 // stage fused into the up-projection.
 cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, void* o, int* err,
                                       int T, int n_h, int d_c, int d_v, bool pdl, cudaStream_t s,

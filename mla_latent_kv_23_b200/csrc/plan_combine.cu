@@ -19,6 +19,7 @@
 //          log-sum-exp: lse = log sum_s exp(lse_s), u = sum_s exp(lse_s - lse) u_s
 //          (the split-KV merge of softmax attention; exact up to rounding).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <limits.h>
 #include <math.h>
 
@@ -263,20 +264,22 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (lse_out != nullptr && lane == 0) lse_out[static_cast<size_t>(br) * n_h + h] = lse_all;
 }
 
-// Merge of the partials with d_c = 512 (the tensor-core path): bf16 or fp32
-// partials, bf16 or fp32 u.  One warp per output row; lane l owns columns
-// [16 l, 16 l + 16).  The partials of up to kGroup splits (8 bf16 or 4 fp32
-// rows: 32 or 64 bytes per lane each) are loaded before any is used, so a
-// row waits for memory about once per group instead of once per split.
-template <bool kOutBf16, bool kPartBf16>
+// Merge of the partials with d_c = 512 (the tensor-core path): bf16, fp16 or
+// fp32 partials (kPart 1, 2, 0), bf16 or fp32 u.  One warp per output row;
+// lane l owns columns [16 l, 16 l + 16).  The partials of up to kGroup splits
+// (8 16-bit or 4 fp32 rows: 32 or 64 bytes per lane each) are loaded before
+// any is used, so a row waits for memory about once per group instead of
+// once per split.
+template <bool kOutBf16, int kPart>
 __global__ void __launch_bounds__(kCombineThreads)
     combine512_kernel(const int* __restrict__ tile_prefix, const int* __restrict__ split_base,
                       const void* __restrict__ part_u, const float* __restrict__ part_lse,
                       void* __restrict__ u_out, float* __restrict__ lse_out, int s_q, int n_h,
                       int rows) {
   constexpr int kDc = 512;
-  constexpr int kGroup = kPartBf16 ? 8 : 4;
-  constexpr int kVecs = kPartBf16 ? 2 : 4;  // 16-byte loads per lane per partial row
+  constexpr bool k16 = kPart != 0;
+  constexpr int kGroup = k16 ? 8 : 4;
+  constexpr int kVecs = k16 ? 2 : 4;  // 16-byte loads per lane per partial row
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   // The tile prefix and split bases come from the plan stage or from the
@@ -305,8 +308,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     for (int k = 0; k < kGroup; ++k) {
       if (s0 + k < nsplit) {
         const size_t e0 = ((slot0 + (size_t)(s0 + k) * s_q) * n_h + h) * kDc + 16 * lane;
-        const uint4* src = kPartBf16
-            ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(part_u) + e0)
+        const uint4* src = k16
+            ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(part_u) + e0)
             : reinterpret_cast<const uint4*>(static_cast<const float*>(part_u) + e0);
 #pragma unroll
         for (int i = 0; i < kVecs; ++i) v[k][i] = src[i];
@@ -343,11 +346,19 @@ __global__ void __launch_bounds__(kCombineThreads)
       for (int k = 0; k < kGroup; ++k) {
         const float w = __shfl_sync(0xffffffffu, w_me, k);
         if (k < n_here) {
-          if (kPartBf16) {
+          if (kPart == 1) {
             const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(v[k]);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float2 f = __bfloat1622float2(x[e]);
+              acc[2 * e] += w * f.x;
+              acc[2 * e + 1] += w * f.y;
+            }
+          } else if (kPart == 2) {
+            const __half2* x = reinterpret_cast<const __half2*>(v[k]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 f = __half22float2(x[e]);
               acc[2 * e] += w * f.x;
               acc[2 * e + 1] += w * f.y;
             }
@@ -407,13 +418,18 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
   const bool out_bf16 = !a.out_f32;
   if (a.d_c == 512) {
     if (a.part_bf16)
-      return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, true>, tp, sb, pu, pl, a.u,
+      return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, 1>, tp, sb, pu, pl, a.u,
                                            a.lse, a.s_q, a.n_h, rows)
-                      : cudaLaunchKernelEx(&cfg, combine512_kernel<false, true>, tp, sb, pu, pl,
+                      : cudaLaunchKernelEx(&cfg, combine512_kernel<false, 1>, tp, sb, pu, pl,
                                            a.u, a.lse, a.s_q, a.n_h, rows);
-    return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, false>, tp, sb, pu, pl, a.u,
+    if (a.part_f16)
+      return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, 2>, tp, sb, pu, pl, a.u,
+                                           a.lse, a.s_q, a.n_h, rows)
+                      : cudaLaunchKernelEx(&cfg, combine512_kernel<false, 2>, tp, sb, pu, pl,
+                                           a.u, a.lse, a.s_q, a.n_h, rows);
+    return out_bf16 ? cudaLaunchKernelEx(&cfg, combine512_kernel<true, 0>, tp, sb, pu, pl, a.u,
                                          a.lse, a.s_q, a.n_h, rows)
-                    : cudaLaunchKernelEx(&cfg, combine512_kernel<false, false>, tp, sb, pu, pl, a.u,
+                    : cudaLaunchKernelEx(&cfg, combine512_kernel<false, 0>, tp, sb, pu, pl, a.u,
                                          a.lse, a.s_q, a.n_h, rows);
   }
   if (out_bf16 && a.part_bf16)

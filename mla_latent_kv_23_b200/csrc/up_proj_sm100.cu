@@ -21,10 +21,11 @@
 //
 // kSplitU can also merge the split-KV partial results itself (the combine
 // of mla_decode, fused in): a row whose sequence was cut into pieces gets
-// lse = log sum_s exp(lse_s) and u = sum_s exp(lse_s - lse) u_s from the fp32
+// lse = log sum_s exp(lse_s) and u = sum_s exp(lse_s - lse) u_s from the fp16
 // partials (written to u and lse as well), a whole row is read as the attend
 // stage wrote it; either way the fp32 row then enters the MMA as hi + lo.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.h"
 #include "sm100_ptx.cuh"
@@ -62,7 +63,7 @@ struct Params {
   int merge, s_q;
   const int* tile_prefix;
   const int* split_base;
-  const float* part_u;
+  const __half* part_u;  // fp16 partial u of split rows
   const float* part_lse;
   float* u_out;        // = u_f32: merged rows are written back
   float* lse_out;      // may be null
@@ -182,18 +183,18 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
         const int nsplit = nsp[j];
         const size_t slot0 = (size_t)sb0[j] * p.s_q + t % p.s_q;  // slot of split s: slot0 + s s_q
         auto lse_of = [&](int sp) { return p.part_lse[(slot0 + (size_t)sp * p.s_q) * p.n_h + head]; };
-        auto part_of = [&](int sp) {
-          return reinterpret_cast<const float4*>(
+        auto part_of = [&](int sp) {  // lane's 16 fp16 values: two 16-byte loads
+          return reinterpret_cast<const uint4*>(
               p.part_u + ((slot0 + (size_t)sp * p.s_q) * p.n_h + head) * 512 + 16 * lane);
         };
         // the first four partial rows are requested together with the
         // statistics: one memory round trip for rows of up to four pieces
-        float4 v[4][4];
+        uint4 v[4][2];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           if (k < nsplit) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[k][i] = part_of(k)[i];
+            for (int i = 0; i < 2; ++i) v[k][i] = part_of(k)[i];
           }
         const float x_lane = lane < nsplit ? lse_of(lane) : -INFINITY;
         float m = x_lane, z = x_lane == -INFINITY ? 0.f : 1.f;
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
               for (int k = 0; k < 4; ++k)
                 if (k < n_here) {
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) v[k][i] = part_of(s0 + k)[i];
+                  for (int i = 0; i < 2; ++i) v[k][i] = part_of(s0 + k)[i];
                 }
             }
 #pragma unroll
@@ -232,11 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
               const float w = s0 + k < 32 ? wk : (k < n_here ? expf(lse_of(s0 + k) - lse) : 0.f);
               if (k < n_here) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  acc[4 * i] += w * v[k][i].x;
-                  acc[4 * i + 1] += w * v[k][i].y;
-                  acc[4 * i + 2] += w * v[k][i].z;
-                  acc[4 * i + 3] += w * v[k][i].w;
+                for (int e = 0; e < 8; ++e) {
+                  const float2 f = __half22float2(reinterpret_cast<const __half2*>(v[k])[e]);
+                  acc[2 * e] += w * f.x;
+                  acc[2 * e + 1] += w * f.y;
                 }
               }
             }
@@ -433,7 +433,7 @@ cudaError_t launch_up_proj_sm100_f32u(const CUtensorMap& w_map, const float* u, 
     p.s_q = merge->s_q;
     p.tile_prefix = merge->tile_prefix;
     p.split_base = merge->split_base;
-    p.part_u = merge->part_u;
+    p.part_u = reinterpret_cast<const __half*>(merge->part_u);
     p.part_lse = merge->part_lse;
     p.u_out = const_cast<float*>(u);
     p.lse_out = merge->lse;

@@ -19,7 +19,7 @@ MLA_DTYPE_BF16 = 0
 MLA_DTYPE_FP32 = 1
 STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_CUDA",
           4: "MLA_ERR_WORKSPACE_TOO_SMALL", 5: "MLA_ERR_DEVICE_CHECK"}
-DEVFLAG_BAD_SEQLEN, DEVFLAG_BAD_PAGE, DEVFLAG_TIMEOUT, DEVFLAG_LAYOUT = 1, 2, 4, 8
+DEVFLAG_BAD_SEQLEN, DEVFLAG_BAD_PAGE, DEVFLAG_TIMEOUT, DEVFLAG_LAYOUT, DEVFLAG_RANGE = 1, 2, 4, 8, 16
 
 
 class MLAError(RuntimeError):

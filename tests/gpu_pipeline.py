@@ -88,20 +88,26 @@ def check_expanded(w, inp, out, picks=None):
 # 2^-8 (abs_v + |o|), abs_v = sum_j a_j |W^UV c_j|, and o's bf16 rounding
 # adds 2^-8 |o|; with an fp32 u the up-projection splits u into two bf16
 # terms (error 2^-16 |u|), with a bf16 u it adds 2^-8 |W^UV| (abs_c + |u|).
+# With an fp32 u the partials of split rows are fp16 (11 significant bits):
+# they add 2^-11 abs_c_k to u and 2^-11 |W^UV| abs_c to o.
 # The checks allow 1.5x these (fp32 accumulation order, the (1 + 2^-7)).
 TIGHT_SLACK = 1.5
 
 
 def tight_u_bound(u_ref, abs_c, u_fp32=True):
     b = 2.0 ** -8 * (abs_c + np.abs(u_ref))
-    if not u_fp32:
+    if u_fp32:
+        b = b + 2.0 ** -11 * abs_c
+    else:
         b = b + 2.0 ** -8 * (abs_c + np.abs(u_ref))
     return TIGHT_SLACK * b + 1e-6
 
 
 def tight_o_bound(o_ref, abs_v, W_i, u_ref, abs_c=None, u_fp32=True):
     b = 2.0 ** -8 * (abs_v + 2.0 * np.abs(o_ref))
-    if not u_fp32:
+    if u_fp32:
+        b = b + 2.0 ** -11 * (np.abs(W_i) @ abs_c)
+    else:
         b = b + 2.0 ** -8 * (np.abs(W_i) @ (abs_c + np.abs(u_ref)))
     return TIGHT_SLACK * b + 1e-6
 

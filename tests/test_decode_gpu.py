@@ -294,6 +294,29 @@ def test_device_flags_for_bad_inputs():
     assert mla.mla_check_device_errors() == 0   # flags were cleared
 
 
+def test_fp16_partials_out_of_range_are_flagged():
+    # with an fp32 u the partial u of a split row is stored in fp16; latent
+    # values beyond its range (here 1e5) raise MLA_DEVFLAG_RANGE, and a
+    # batch within range raises nothing
+    w = v3_small(B=1, seqlens=(700,), block_table="identity")
+    inp = synth.draw(w)
+    q = to_dev(synth.random_q(w), w)
+    bt, sl = to_dev_i32(inp["block_table"]), to_dev_i32(inp["seqlens"])
+    cache = to_dev(inp["cache"], w)
+    mla.decode(q, cache, bt, sl, w.page_size, w.d_R, w.softmax_scale, 4)
+    assert mla.mla_check_device_errors() == 0
+    big = cache.clone()
+    big[:, :w.d_c] *= 1e5
+    mla.decode(q, big, bt, sl, w.page_size, w.d_R, w.softmax_scale, 4)
+    with pytest.raises(mla.MLAError) as e:
+        mla.mla_check_device_errors()
+    assert e.value.flags & mla.DEVFLAG_RANGE
+    # one chunk: the row is written whole in fp32, nothing to flag
+    u, _ = mla.decode(q, big, bt, sl, w.page_size, w.d_R, w.softmax_scale, 1)
+    assert mla.mla_check_device_errors() == 0
+    assert torch.isfinite(u).all()
+
+
 def test_bounded_wait_gives_up_and_the_context_stays_usable():
     # the wait every kernel uses on its mbarriers: on a phase that completes
     # it returns at once; on one that never completes it gives up after its
