@@ -261,7 +261,7 @@ def run_gpu(args, w):
     q0, W_QK = absorb_and_query(wr, inp, dev)
     del W_QK
     cache_bytes = inp["num_pages"] * w.page_size * w.width * 2
-    step_in_bytes = cache_bytes + q0.numel() * 2
+    step_in_bytes = cache_bytes + q0.numel() * 2 + w.n_h * w.d_v * w.d_c * 2  # + W^UV
     R = max(2, math.ceil(3 * L2_BYTES / step_in_bytes))
     caches = [torch.from_numpy(inp["cache"]).to(dev).to(tdt)]
     for _ in range(R - 1):
@@ -270,6 +270,9 @@ def run_gpu(args, w):
     bt = torch.from_numpy(inp["block_table"]).to(dev)
     sl = torch.from_numpy(inp["seqlens"]).to(dev)
     W_UV = torch.from_numpy(inp["W_UV"]).to(dev).to(tdt)
+    # the weights rotate with the inputs: a decode loop reads another layer's W^UV
+    # between two uses of one layer's, so no step finds them in L2 from the last
+    W_UVs = [W_UV] + [W_UV.clone() for _ in range(R - 1)]
     T = w.B * w.s_q
     u = torch.empty((w.B, w.s_q, w.n_h, w.d_c), dtype=udt, device=dev)
     lse = torch.empty((w.B, w.s_q, w.n_h), dtype=torch.float32, device=dev)
@@ -292,7 +295,7 @@ def run_gpu(args, w):
         p = params[i % R]
         if ev is None:
             if fused:
-                mla.mla_decode_step(p, W_UV, o, ws)
+                mla.mla_decode_step(p, W_UVs[i % R], o, ws)
                 return
             mla.mla_decode(p, ws)
         else:
@@ -303,7 +306,7 @@ def run_gpu(args, w):
             ev[1].record()
             mla.mla_decode_combine(p, ws)
             ev[3].record()
-        mla.mla_up_proj(u.view(T, w.n_h, w.d_c), W_UV, o)
+        mla.mla_up_proj(u.view(T, w.n_h, w.d_c), W_UVs[i % R], o)
 
     # direct launches once (initialises the library, checks flags)
     stream = torch.cuda.Stream(device=dev)
