@@ -137,7 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
   if constexpr (kMode == UpMode::kSplitU) {
    if (p.merge) {
     // One warp per row t (rows warp and warp + 16 of the block); lane l
-    // owns columns [16 l, 16 l + 16) of d_c = 512.  The plan stage's
+    // owns columns [8 l, 8 l + 8) and [256 + 8 l, 256 + 8 l + 8) of
+    // d_c = 512, so each 16-byte access of the warp covers 512 contiguous
+    // bytes of a row (one fp16 partial row or half an fp32 row).  The plan stage's
     // outputs are read before the wait: the plan kernel completed before
     // the attend kernel passed its own wait, and this kernel was launched
     // only after every attend CTA had passed it.
@@ -168,24 +170,25 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0.f;
       const size_t urow = (size_t)t * p.n_h + head;
-      float* up = p.u_out + urow * 512 + 16 * lane;
+      float* up = p.u_out + urow * 512 + 8 * lane;  // float4 i of the lane: up + 256 (i >> 1) + 4 (i & 1)
       if (kind[j] == 1) {  // written whole by the attend stage
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float4 v = reinterpret_cast<const float4*>(up)[i];
+          const float4 v = reinterpret_cast<const float4*>(up + (i >> 1) * 256)[i & 1];
           acc[4 * i] = v.x; acc[4 * i + 1] = v.y; acc[4 * i + 2] = v.z; acc[4 * i + 3] = v.w;
         }
       } else if (kind[j] == 2) {  // no tokens (a rejected length): u = 0, lse = -inf
 #pragma unroll
-        for (int i = 0; i < 4; ++i) reinterpret_cast<float4*>(up)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(up + (i >> 1) * 256)[i & 1] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (lane == 0 && p.lse_out) p.lse_out[urow] = -INFINITY;
       } else if (kind[j] == 3) {
         const int nsplit = nsp[j];
         const size_t slot0 = (size_t)sb0[j] * p.s_q + t % p.s_q;  // slot of split s: slot0 + s s_q
         auto lse_of = [&](int sp) { return p.part_lse[(slot0 + (size_t)sp * p.s_q) * p.n_h + head]; };
-        auto part_of = [&](int sp) {  // lane's 16 fp16 values: two 16-byte loads
+        auto part_of = [&](int sp) {  // lane's 16 fp16 values: 16-byte elements 0 and 32
           return reinterpret_cast<const uint4*>(
-              p.part_u + ((slot0 + (size_t)sp * p.s_q) * p.n_h + head) * 512 + 16 * lane);
+              p.part_u + ((slot0 + (size_t)sp * p.s_q) * p.n_h + head) * 512 + 8 * lane);
         };
         // the first four partial rows are requested together with the
         // statistics: one memory round trip for rows of up to four pieces
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
         for (int k = 0; k < 4; ++k)
           if (k < nsplit) {
 #pragma unroll
-            for (int i = 0; i < 2; ++i) v[k][i] = part_of(k)[i];
+            for (int i = 0; i < 2; ++i) v[k][i] = part_of(k)[32 * i];
           }
         const float x_lane = lane < nsplit ? lse_of(lane) : -INFINITY;
         float m = x_lane, z = x_lane == -INFINITY ? 0.f : 1.f;
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
               for (int k = 0; k < 4; ++k)
                 if (k < n_here) {
 #pragma unroll
-                  for (int i = 0; i < 2; ++i) v[k][i] = part_of(s0 + k)[i];
+                  for (int i = 0; i < 2; ++i) v[k][i] = part_of(s0 + k)[32 * i];
                 }
             }
 #pragma unroll
@@ -244,16 +247,17 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          reinterpret_cast<float4*>(up)[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+          reinterpret_cast<float4*>(up + (i >> 1) * 256)[i & 1] =
+              make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
         if (lane == 0 && p.lse_out) p.lse_out[urow] = lse;
       }
-      // the row's two bf16 terms: lane l's 16 columns are chunks 2l, 2l + 1
+      // the row's two bf16 terms: lane l's 16 columns are chunks l, 32 + l
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float v8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) v8[k] = acc[8 * c + k];
-        store_hilo(tt, 2 * lane + c, v8);
+        store_hilo(tt, lane + 32 * c, v8);
       }
     }
     fence_proxy_async_smem();
@@ -342,7 +346,27 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
         for (int k = 0; k < 32; ++k) d[k] += e[k];
       }
       tmem_wait_ld();
-      if (v < p.d_v) {
+      if (kMode == UpMode::kSplitU && p.d_v % 8 == 0) {
+        // rows [c0, c0 + 32) go through the B-operand area (free once the
+        // product is complete) as [t][v] bf16, then leave as 16-byte
+        // stores of 8 consecutive v: one 2-byte store per value backs up
+        // behind the merge's stores of u
+        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(base + off_u);
+        if (v < p.d_v) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (c0 + k < p.n_pad) stg[k * kM + v] = __float2bfloat16_rn(d[k]);
+        }
+        named_bar_sync(1, 4 * 32);
+        const int rows = min(32, p.n_pad - c0), per_row = p.d_v / 8;
+        for (int i = threadIdx.x; i < rows * per_row; i += 4 * 32) {
+          const int k = i / per_row, v8 = 8 * (i % per_row), t = t0 + c0 + k;
+          if (t < p.T)
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + ((size_t)t * p.n_h + head) * p.d_v + v8) =
+                *reinterpret_cast<const uint4*>(stg + k * kM + v8);
+        }
+        named_bar_sync(1, 4 * 32);  // the area is read before the next rows land in it
+      } else if (v < p.d_v) {
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           const int t = t0 + c0 + k;
