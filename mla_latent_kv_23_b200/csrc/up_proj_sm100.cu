@@ -134,6 +134,13 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
     st_shared_v4(blk + tt * 128 + sw, hi[0], hi[1], hi[2], hi[3]);
     st_shared_v4(blk + (p.n_pad + tt) * 128 + sw, lo[0], lo[1], lo[2], lo[3]);
   };
+  // merged rows of split sequences, kept in registers until the product has
+  // been issued: it reads only their bf16 terms in shared memory
+  constexpr int kKeep = kMode == UpMode::kSplitU ? kMaxRowsSplit / (kThreads / 32) : 1;
+  float keep_u[kKeep][16], keep_lse[kKeep];
+  bool keep[kKeep];
+#pragma unroll
+  for (int j = 0; j < kKeep; ++j) keep[j] = false;
   if constexpr (kMode == UpMode::kSplitU) {
    if (p.merge) {
     // One warp per row t (rows warp and warp + 16 of the block); lane l
@@ -246,10 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
           }
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          reinterpret_cast<float4*>(up + (i >> 1) * 256)[i & 1] =
-              make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-        if (lane == 0 && p.lse_out) p.lse_out[urow] = lse;
+        for (int i = 0; i < 16; ++i) keep_u[j][i] = acc[i];
+        keep_lse[j] = lse;
+        keep[j] = true;
       }
       // the row's two bf16 terms: lane l's 16 columns are chunks l, 32 + l
 #pragma unroll
@@ -327,8 +333,21 @@ __global__ void __launch_bounds__(kThreads, 1) up_proj_sm100_kernel(const __grid
           }
     }
     umma_commit(bar_mma);
-    if (!mbar_wait(bar_mma, 0, p.err, MLA_DEVFLAG_TIMEOUT)) ok = false;
   }
+  if constexpr (kMode == UpMode::kSplitU) {  // the merged rows leave while the product runs
+#pragma unroll
+    for (int j = 0; j < kKeep; ++j)
+      if (keep[j]) {
+        const size_t urow = (size_t)(t0 + warp + j * (kThreads / 32)) * p.n_h + head;
+        float* up = p.u_out + urow * 512 + 8 * lane;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(up + (i >> 1) * 256)[i & 1] =
+              make_float4(keep_u[j][4 * i], keep_u[j][4 * i + 1], keep_u[j][4 * i + 2], keep_u[j][4 * i + 3]);
+        if (lane == 0 && p.lse_out) p.lse_out[urow] = keep_lse[j];
+      }
+  }
+  if (threadIdx.x == 0 && !mbar_wait(bar_mma, 0, p.err, MLA_DEVFLAG_TIMEOUT)) ok = false;
   ok = __syncthreads_and(ok);
   tc_fence_after();
   if (ok && warp < 4) {
