@@ -190,12 +190,13 @@ def test_running_max_jumps_across_tiles(s_q, splits):
     assert_tight(check_absorbed(w, q, inp, out, picks, W_UV=inp["W_UV"]))
 
 
-@pytest.mark.parametrize("T", [1, 16, 33, 100])
-def test_up_projection_of_fp32_u(T):
+@pytest.mark.parametrize("T,d_v", [(1, 128), (16, 128), (33, 128), (100, 128), (17, 40), (16, 100), (3, 12)])
+def test_up_projection_of_fp32_u(T, d_v):
     # an fp32 u (spread up to ~|u| 25 like the stress workload) against the
     # exact product: the two bf16 terms of u leave 2^-16 |u|, so only o's own
-    # bf16 rounding (2^-8 |o|) and fp32 accumulation remain
-    w = v3_small(B=T, seqlens=(1,) * T, block_table="identity")
+    # bf16 rounding (2^-8 |o|) and fp32 accumulation remain.  d_v below 128
+    # (a multiple of 8: o leaves as 16-byte stores; else one value per store)
+    w = v3_small(B=T, seqlens=(1,) * T, block_table="identity", d_v=d_v)
     inp = synth.draw(w)
     u = (np.random.default_rng(T).standard_normal((T, w.n_h, w.d_c)) * 8).astype(np.float32)
     W_UV = to_dev(inp["W_UV"], w)
@@ -433,12 +434,13 @@ def test_merge_partials_against_its_definition(dtype, d_c, R):
     assert err.max() <= tol
 
 
-@pytest.mark.parametrize("s_q,splits", [(1, 0), (1, 5), (2, 0), (2, 3)])
-def test_decode_step_fuses_the_combine_into_the_up_projection(s_q, splits):
+@pytest.mark.parametrize("s_q,splits,d_v", [(1, 0, 128), (1, 5, 128), (2, 0, 128), (2, 3, 128),
+                                           (1, 5, 40), (2, 3, 100)])
+def test_decode_step_fuses_the_combine_into_the_up_projection(s_q, splits, d_v):
     # mla_decode_step merges split rows inside the up-projection; it returns
     # what mla_decode followed by mla_up_proj returns, bit for bit (the same
     # arithmetic in the same order), and meets the oracle's bounds
-    w = v3_small(s_q=s_q, B=5, seqlens=(100, 1000, 777, 64, 2))
+    w = v3_small(s_q=s_q, B=5, seqlens=(100, 1000, 777, 64, 2), d_v=d_v)
     inp = synth.draw(w)
     q = synth.random_q(w)
     qd, cache = to_dev(q, w), to_dev(inp["cache"], w)
