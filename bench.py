@@ -79,10 +79,19 @@ def load_peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0), "fallback"
 
 
+def code_only(text: str) -> str:
+    """Source text without comments, trailing blanks and empty lines: a
+    change to comments alone leaves the compiled kernel and its hash as they
+    were."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, "mla_latent_kv_23_b200", "csrc", f), "rb").read())
+        h.update(code_only(open(os.path.join(ROOT, "mla_latent_kv_23_b200", "csrc", f)).read()).encode())
     return h.hexdigest()[:16]
 
 

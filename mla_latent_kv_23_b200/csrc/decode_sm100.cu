@@ -50,11 +50,15 @@
 // (even CTA only); warp 3 = relay: loads the segment's query by TMA,
 // zeroes cache rows past a sequence's end in this CTA's stage, and signals
 // the even CTA's barriers that this CTA's operands are in place; warps 4-11
-// = softmax: warp 4 + 4c + q reads TMEM lanes [32q, 32q + 32) and tokens
-// [32c, 32c + 32) of a tile.  Each thread finishes 16 scores of one head; the
-// row maximum is shared through shared memory with one 8-warp rendezvous per
-// tile.  O rows are rescaled by the warp that can reach their TMEM lanes,
-// which derives the same maximum from the same shared values.
+// = softmax, two groups of four: group g takes the tiles whose S lands in S
+// buffer g (every other tile), and warp 4 + 4g + q of it reads TMEM lanes
+// [32q, 32q + 32) of that buffer.  Each thread adds the two column-half
+// partials of one head's scores and finishes 32 of them (tokens
+// [16j, 16j + 16) of each 32-token half, j = lane / 16); the group shares the
+// tile's row maxima through shared memory behind a 4-warp named barrier, and
+// a tile's running-maximum decision waits for the previous tile's, published
+// by the other group.  O rows are rescaled by the warp that can reach their
+// TMEM lanes, which reads the same published maxima.
 //
 // Epilogue: u = O / l leaves TMEM through the query area (free once the
 // segment's last S is done) by TMA stores of whole 128-byte lines; the relay
