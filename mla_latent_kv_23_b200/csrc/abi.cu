@@ -392,7 +392,7 @@ WsLayout ws_layout(int B, int s_q, int n_h, int d_c, int num_chunks) {
   L.chunk_t = off;
   off = align_up(off + sizeof(int) * (num_chunks + 1), 256);
   L.chunk_b = off;
-  off = align_up(off + sizeof(int) * 2 * (size_t)num_chunks, 256);
+  off = align_up(off + sizeof(int) * 4 * (size_t)num_chunks, 256);
   L.part_lse = off;
   off = align_up(off + sizeof(float) * (size_t)L.slots * n_h, 256);
   L.part_u = off;

@@ -25,9 +25,10 @@ constexpr int kSegCostTiles = 4;
 // start, [5] 1 when the chunks follow the sequences (see the plan kernel),
 // [6] the chunks in use (the others are empty).
 // chunk_t[c] is the first tile of chunk c (chunk_t[chunks] = total tiles);
-// chunk_b[2 c] is the sequence that tile belongs to and chunk_b[2 c + 1] the
-// index of that piece among its sequence's pieces (0 when the chunk starts at
-// the sequence's first tile).
+// chunk_b[4 c .. 4 c + 3] is chunk c's record: the sequence that tile belongs
+// to, the index of that piece among its sequence's pieces (0 when the chunk
+// starts at the sequence's first tile), and that sequence's first and end
+// tile on the line (16-byte aligned, one load).
 struct WsLayout {
   size_t header = 0, tile_prefix = 0, split_base = 0, chunk_t = 0, chunk_b = 0, part_lse = 0,
          part_u = 0, total = 0;

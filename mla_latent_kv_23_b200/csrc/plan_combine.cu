@@ -1,8 +1,8 @@
 // Plan and combine stages of mla_decode.
 //
 // plan:    per-sequence tile counts and their prefix sum; the cut of the tile
-//          line into KV chunks; the first tile, sequence and piece index of
-//          every chunk; and the first partial row of every sequence that is
+//          line into KV chunks; the first tile, sequence, piece index and
+//          that sequence's tile range of every chunk; and the first partial row of every sequence that is
 //          cut into several chunks (one block; B is small).  Two cuts:
 //          * aligned: when every sequence has the same tile count t and the
 //            chunks divide among the sequences (c = chunks / B pieces each),
@@ -139,10 +139,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int* __restric
       }
     }
     chunk_t[c] = t;
-    if (c < num_chunks) {
-      chunk_b[2 * c] = sb;
-      chunk_b[2 * c + 1] = part;
-    }
+    if (c < num_chunks)  // the record: sequence, piece, and the sequence's tiles on the line
+      *reinterpret_cast<int4*>(chunk_b + 4 * c) =
+          make_int4(sb, part, sb < B ? tp[sb] : T, sb < B ? tp[sb + 1] : T);
   }
   carry = 0;
   for (int base = 0; base < B; base += blockDim.x) {

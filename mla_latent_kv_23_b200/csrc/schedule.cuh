@@ -24,10 +24,13 @@ struct ChunkWalk {
   const int* tp;  // tile_prefix, B + 1 entries
   int B;
   int t, t_end, b;
-  int part0;  // piece index of the chunk's first segment
+  int part0;            // piece index of the chunk's first segment
+  int b0_begin, b0_end; // tiles [b0_begin, b0_end) of the line: the first segment's sequence
 
-  // chunk_t / chunk_b come from the plan stage; the reads are independent
-  // (one memory round trip)
+  // chunk_t and the chunk's record (sequence, piece, and that sequence's
+  // first and end tile on the line) come from the plan stage; the reads are
+  // independent (one memory round trip), and the first segment needs no
+  // read of the tile prefix
   __device__ __forceinline__ void init(const int* tile_prefix, const int* chunk_t,
                                        const int* chunk_b, const int* header, int nseq,
                                        int chunk_id) {
@@ -36,15 +39,25 @@ struct ChunkWalk {
     B = nseq;
     t = chunk_t[chunk_id];
     t_end = chunk_t[chunk_id + 1];
-    b = chunk_b[2 * chunk_id];
-    part0 = chunk_b[2 * chunk_id + 1];
+    const int4 r = *reinterpret_cast<const int4*>(chunk_b + 4 * chunk_id);
+    b = r.x;
+    part0 = r.y;
+    b0_begin = r.z;
+    b0_end = r.w;
   }
 
   __device__ __forceinline__ bool next(Segment& s) {
     if (t >= t_end) return false;
-    while (b < B && tp[b + 1] <= t) ++b;  // skip sequences that end at or before t
-    if (b >= B) return false;
-    const int begin = tp[b], end = tp[b + 1];
+    int begin, end;
+    if (b < B && t >= b0_begin && t < b0_end) {  // still inside the first segment's sequence
+      begin = b0_begin;
+      end = b0_end;
+    } else {
+      while (b < B && tp[b + 1] <= t) ++b;  // skip sequences that end at or before t
+      if (b >= B) return false;
+      begin = tp[b];
+      end = tp[b + 1];
+    }
     const int stop = min(t_end, end);
     s.b = b;
     s.t0 = t - begin;
