@@ -17,8 +17,10 @@ constexpr int kMaxHeads = 128;    // query heads packed as the MMA M dimension
 // Cost of starting one more sequence inside a KV chunk (loading its queries,
 // writing its output), in units of one 64-token tile.  The plan cuts chunks on
 // a line where every sequence start takes this many units on top of its tiles,
-// so chunks that hold several sequences get fewer tiles.
-constexpr int kSegCostTiles = 4;
+// so chunks that hold several sequences get fewer tiles.  A second segment in
+// a chunk costs the attend kernel about 6-8 us (epilogue, query load,
+// pipeline refill), 5-6 tiles at 1.3-1.4 us each.
+constexpr int kSegCostTiles = 6;
 
 // Workspace of mla_decode.  Header ints: [0] total tiles, [1] line units per
 // chunk, [2] number of chunks, [3] split rows in use, [4] units per sequence
