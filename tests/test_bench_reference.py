@@ -34,3 +34,16 @@ def test_warmup_below_three_is_refused():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
                           "--warmup", "2"], cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_profiled_traffic_is_keyed_to_code_not_comments():
+    # the committed ncu summaries name the attend kernel's code by a hash of
+    # its sources without comments: a comment edit keeps the counters valid,
+    # a code edit drops them (traffic: null) until the kernel is profiled again
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.code_only("int a; // note\n/* block\n comment */ int b;  \n\n  \nint c;") == \
+        "int a;\n int b;\nint c;"
+    assert bench.code_only("x = 1;\n") != bench.code_only("x = 2;\n")
+    h = bench.kernel_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
