@@ -218,7 +218,7 @@ mla_status mla_decode(const mla_decode_params* p, void* workspace, size_t worksp
  * separately; calling them in this order is exactly mla_decode.
  *   plan:    per-sequence tile counts and KV-chunk boundaries into the workspace
  *   attend:  the chunked attention (writes u/lse directly for unsplit rows,
- *            partials into the workspace otherwise, in the type of u)
+ *            partials into the workspace otherwise: see u_fp32 for their type)
  *   combine: merges the partials of split rows into u/lse
  * Called on their own, the stages launch as plain stream-ordered kernels;
  * inside mla_decode each stage may start its prologue while the previous
